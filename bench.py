@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Throughput of the HARP rotate + quantize path on B200.
+
+Workload (the headline configuration): a 4096 x 4096 bf16 weight (Student-t
+nu = 3 entries x 0.02, 0.5 % of input channels x 20), two-sided processor
+(16,16,16) x (16,16,16) with random orthogonal blocks and random signs,
+Lloyd-Max N(0,1) codebooks with group 128 at 2 and at 4 bits.
+
+One step = the whole hot path over that weight, for each bit width:
+rotate + quantize + pack (column kernel, then fused row kernel), then
+dequantize + unrotate (row kernel, then column kernel): 8 kernel launches.
+value = algorithmic bytes of the step (bf16 weight read and codes + fp16
+scales written by each forward; codes + scales read and the bf16 weight
+written by each inverse) / device time, in GB/s. The fp32 intermediate
+between the column and row passes is implementation traffic and is not
+credited. L2 is flushed (512 MB write) before every timed step.
+
+--impl reference times the float64 oracle (the CPU statement of the same
+computation) on the host cores instead, on a bounded sample of the same
+workload. Under torchrun every rank runs an independent replica (the path has
+no exchange step); the time is the maximum over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "rotate+quantize GB/s and % of B200 HBM peak (4096×4096 bf16, two-sided)"
+ROWS = COLS = 4096
+RADIX = (16, 16, 16)
+BITS = (2, 4)
+GROUP = 128
+L2_FLUSH_BYTES = 512 << 20
+WORKLOAD = ("4096x4096 bf16 weight (Student-t nu=3 x0.02, 0.5% input channels x20), two-sided "
+            "HARP processor (16,16,16)x(16,16,16), random orthogonal blocks + random signs; "
+            "Lloyd-Max N(0,1) group 128 at 2 and 4 bits; step = rotate+quantize then "
+            "dequantize+unrotate for each bit width")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
+
+
+def fwd_bytes_per_elem(bits):
+    return 2.0 + bits / 8.0 + 2.0 / GROUP
+
+
+def inv_bytes_per_elem(bits):
+    return bits / 8.0 + 2.0 / GROUP + 2.0
+
+
+STEP_BYTES = ROWS * COLS * sum(fwd_bytes_per_elem(b) + inv_bytes_per_elem(b) for b in BITS)
+FLOP_PER_ELEM_SIDE = 2 * sum(RADIX)      # one FMA per block coefficient per element
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fp32_peak_tflops(sm_mhz):
+    """FFMA peak: 148 SMs x 128 fp32 lanes x 2 flop x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import rotation_preconditioned_bit_b200 as harp
+    from rotation_preconditioned_bit_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.workload("c2")
+    left = harp.Plan.from_side(w.left)
+    right = harp.Plan.from_side(w.right)
+    cbs = [harp.Codebook("lloyd_max", b, GROUP) for b in BITS]
+    x_host = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x = x_host.to(dev)
+    ws = torch.empty((ROWS, COLS), dtype=torch.float32, device=dev)
+    out = torch.empty((ROWS, COLS), dtype=torch.bfloat16, device=dev)
+    outs = [harp.empty_codes(ROWS, COLS, cb, dev) for cb in cbs]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # one step through the single-kernel entry points, events between launches
+    # (the same four kernels the two-sided calls launch, in the same order)
+    names = ["col_fwd", "row_fwd_quant", "row_deq_inv", "col_inv"]
+    kt = {f"{n}_{b}bit": [] for b in BITS for n in names}
+
+    def step(record):
+        evs = []
+        for cb, (codes, scales) in zip(cbs, outs):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
+            if record:
+                e[0].record(stream)
+            harp.harp_rotate(left, harp.HARP_LEFT, harp.HARP_FWD, x, ws, stream)
+            if record:
+                e[1].record(stream)
+            harp.harp_rotate_quantize(None, right, cb, ws, codes, scales, None, None, stream)
+            if record:
+                e[2].record(stream)
+            harp.harp_dequantize_unrotate(None, right, cb, codes, scales, ws, None, stream)
+            if record:
+                e[3].record(stream)
+            harp.harp_rotate(left, harp.HARP_LEFT, harp.HARP_INV, ws, out, stream)
+            if record:
+                e[4].record(stream)
+                evs.append((cb.bits, e))
+        return evs
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    step_ms = []
+    all_evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        evs = step(True)
+        s1.record(stream)
+        all_evs.append((s0, s1, evs))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    for s0, s1, evs in all_evs:
+        step_ms.append(s0.elapsed_time(s1))
+        for bits, e in evs:
+            for i, n in enumerate(names):
+                kt[f"{n}_{bits}bit"].append(e[i].elapsed_time(e[i + 1]))
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = t.item()
+        torch.distributed.barrier()
+
+    # ---- end to end through the public two-sided calls, host buffers
+    e2e = None
+    if not args.no_e2e:
+        codes_h = [torch.empty(c.shape, dtype=c.dtype).pin_memory() for c, _ in outs]
+        scales_h = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for _, s in outs]
+        out_h = torch.empty((ROWS, COLS), dtype=torch.bfloat16).pin_memory()
+        h2d = x_host.numel() * 2
+        d2h = sum(c.numel() + s.numel() * 2 + out_h.numel() * 2 for c, s in outs)
+        ws_bytes = ws.numel() * 4
+
+        def e2e_step():
+            x.copy_(x_host, non_blocking=True)
+            for i, (cb, (codes, scales)) in enumerate(zip(cbs, outs)):
+                harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws, stream)
+                codes_h[i].copy_(codes, non_blocking=True)
+                scales_h[i].copy_(scales, non_blocking=True)
+                harp.harp_dequantize_unrotate(left, right, cb, codes, scales, out, ws, stream)
+                out_h.copy_(out, non_blocking=True)
+
+        for _ in range(max(2, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e_ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            b.synchronize()
+            e_ms.append(a.elapsed_time(b))
+        e_total = sum(e_ms)
+        if world > 1:
+            t = torch.tensor([e_total], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_total = t.item()
+        e2e = {"value": round(world * STEP_BYTES * args.steps / (e_total * 1e-3) / 1e9, 2),
+               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_total / args.steps, 4),
+               "api": "harp_rotate_quantize + harp_dequantize_unrotate (two-sided), pinned host buffers",
+               "workspace_bytes": ws_bytes}
+    del flush
+    return total_ms, step_ms, kt, clk, e2e
+
+
+def kernel_table(kt):
+    n = ROWS * COLS
+    out = {}
+    for key, v in kt.items():
+        if not v:
+            continue
+        us = 1e3 * statistics.mean(v)
+        name, bits = key.rsplit("_", 1)
+        b = int(bits[:-3])
+        if name == "col_fwd":
+            alg = n * 2.0                      # bf16 weight in (fp32 intermediate not credited)
+            own = n * (2.0 + 4.0)
+        elif name == "row_fwd_quant":
+            alg = n * (b / 8.0 + 2.0 / GROUP)  # codes + scales out
+            own = n * (4.0 + b / 8.0 + 2.0 / GROUP)
+        elif name == "row_deq_inv":
+            alg = n * (b / 8.0 + 2.0 / GROUP)
+            own = n * (b / 8.0 + 2.0 / GROUP + 4.0)
+        else:
+            alg = n * 2.0
+            own = n * (4.0 + 2.0)
+        flop = n * FLOP_PER_ELEM_SIDE
+        out[key] = {"us": round(us, 2), "own_bytes": int(own), "own_gbs": round(own / (us * 1e-6) / 1e9, 1),
+                    "alg_bytes": int(alg), "tflops": round(flop / (us * 1e-6) / 1e12, 2)}
+    return out
+
+
+# ------------------------------------------------------------ CPU (oracle) arm
+
+_C2 = {}
+
+
+def _c2_oracle_inputs():
+    if not _C2:
+        import oracle
+        from rotation_preconditioned_bit_b200 import synth
+        w = synth.workload("c2")
+        _C2["X"] = synth.x_as_f64(w)
+        _C2["P"] = (oracle.processor(w.left), oracle.processor(w.right))
+    return _C2["X"], _C2["P"]
+
+
+def oracle_sample(frac):
+    """The float64 oracle on a sample of the step: the left pass on a column
+    strip and the right pass + quantise + inverse on a row strip, each a
+    fraction `frac` of the weight, for the 2-bit variant. Returns (seconds,
+    algorithmic bytes credited, description)."""
+    import oracle
+
+    X, (Pl, Pr) = _c2_oracle_inputs()
+    nc = max(1, int(round(COLS * frac)))
+    nr = max(1, int(round(ROWS * frac)))
+    bits = BITS[0]
+    t0 = time.perf_counter()
+    T = Pl.rotate_cols(X[:, :nc])
+    Y = Pr.rotate_rows(X[:nr, :])
+    codes, scales, _, _ = oracle.quantize("lloyd_max", bits, GROUP, Y, with_margins=False)
+    packed = oracle.pack(bits, codes)
+    codes2 = oracle.unpack(bits, packed, COLS)
+    Yh = oracle.dequantize("lloyd_max", bits, GROUP, codes2, scales)
+    Z = Pr.rotate_rows(Yh, inverse=True)
+    U = Pl.rotate_cols(T, inverse=True)
+    dt = time.perf_counter() - t0
+    del T, Z, U
+    elems = nc * ROWS                              # both sides cover this many elements
+    credited = elems * (fwd_bytes_per_elem(bits) + inv_bytes_per_elem(bits))
+    desc = (f"float64 oracle, 2-bit variant: left pass on a {ROWS}x{nc} column strip and right pass "
+            f"+ quantise + pack + dequantise + inverse on a {nr}x{COLS} row strip "
+            f"({frac:.3f} of the weight), single thread")
+    return dt, credited, desc
+
+
+def pick_frac(budget_s):
+    dt, _, _ = oracle_sample(1.0 / 64)
+    per_full = dt * 64
+    return max(1.0 / 256, min(1.0, budget_s / per_full))
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    budget = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    frac = pick_frac(budget)
+    for _ in range(args.warmup):
+        oracle_sample(frac)
+    secs, credited, desc = 0.0, 0.0, ""
+    for _ in range(args.steps):
+        dt, cr, desc = oracle_sample(frac)
+        secs += dt
+        credited += cr
+    value = credited / secs / 1e9
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * secs / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "parallelism": "replicas", "l2": "n/a (host)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="harp", choices=["harp", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    total_ms, step_ms, kt, clk, e2e = run_gpu(args, rank, world, local_rank)
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        value = world * STEP_BYTES * args.steps / (total_ms * 1e-3) / 1e9
+        ktab = kernel_table(kt)
+        # dominant kernel: largest total time in the step
+        dom = max(ktab, key=lambda k: ktab[k]["us"])
+        smhz = float(peaks.get("sm_max_mhz", 1965.0))
+        peak_tf = fp32_peak_tflops(smhz)
+        d = ktab[dom]
+        roof = {"kernel": dom, "bound": "alu", "achieved": d["tflops"], "peak": round(peak_tf, 1),
+                "unit": "TFLOP/s", "frac": round(d["tflops"] / peak_tf, 4), "traffic": None,
+                "peak_source": f"FFMA: 148 SM x 128 lanes x 2 flop x {smhz:.0f} MHz (max SM clock, {peak_src})",
+                "algorithmic": f"{FLOP_PER_ELEM_SIDE} flop per element per side ({sum(RADIX)} FMA)",
+                "own_bytes_hbm_frac": round(d["own_gbs"] / hbm, 4)}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            frac = pick_frac(args.cpu_budget)
+            dt, credited, desc = oracle_sample(frac)
+            cpu = {"value": round(credited / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": desc, "seconds": round(dt, 2)}
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "in_dtype": "bf16",
+                           "left_radix": list(RADIX), "right_radix": list(RADIX), "bits": list(BITS),
+                           "group": GROUP, "parallelism": "replicas" if world > 1 else "single",
+                           "l2": "flushed before every timed step (512 MB write)",
+                           "step_bytes": int(STEP_BYTES)},
+                "hbm_frac": round(value / world / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": peak_src,
+                "roofline": roof, "kernels": ktab, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 8 * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

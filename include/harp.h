@@ -1,0 +1,236 @@
+/*
+ * harp.h -- C ABI of libharp: HARP's structured orthogonal processor fused
+ * with a group-wise low-bit quantizer, on one NVIDIA B200 (sm_100a).
+ *
+ * What it computes (the pages' titles and sections):
+ *  - HARP: Hadamard-Preconditioned Adaptive Rotation Processor for Extreme
+ *    LLM Quantization (gist.science, paper 2605.29843), section 2.1: a
+ *    processor on R^d is a product of m stride stages with mixed radices
+ *    b_0 .. b_{m-1}, prod b_t = d; stage t applies one b_t x b_t orthogonal
+ *    block to each group of coordinates that a stride permutation separates.
+ *    Section 2.2: blocks B = Q(theta) G_b, G_b a normalised Sylvester
+ *    Hadamard (b = 2^k) or the Q factor of a fixed Gaussian; theta = 0 gives
+ *    the fixed randomized Hadamard transform (random signs, then Hadamard).
+ *    Sections 3 and 5: two-sided on weights (W' = U^T W V), one-sided on
+ *    activations; an exact change of basis, undone by the transpose.
+ *  - PolarQuant: Optimal Gaussian Weight Quantization via Hadamard Rotation
+ *    for LLM Compression (gist.science, paper 2603.29078), section 2:
+ *    rotated groups scaled to N(0,1) and coded with Lloyd-Max centroids;
+ *    fp16 group scale, fp32 centroid table; section 1: the absmax uniform
+ *    quantizer on [-alpha, alpha].
+ *
+ * Conventions fixed by this library where the pages leave them open:
+ *  - Index convention. s_t = b_{t+1} * ... * b_{m-1} (s_{m-1} = 1). Stage t's
+ *    group c = h*s_t + l (0 <= l < s_t) holds the coordinates
+ *    h*b_t*s_t + k*s_t + l, k = 0 .. b_t-1, and
+ *        y[h b s + k s + l] = sum_j B_{t,c}[k][j] * x[h b s + j s + l].
+ *    The processor is M = B_{m-1} ... B_1 B_0 D_s: the sign vector first,
+ *    then stage 0 (largest stride). Its inverse is D_s B_0^T ... B_{m-1}^T.
+ *  - Sides. HARP_RIGHT maps every row r of a [rows x cols] matrix to M r
+ *    (d = cols; X -> X V with V = M^T). HARP_LEFT maps every column w to M w
+ *    (d = rows; W -> U^T W with U = M^T). Two-sided: W' = M_L W M_R^T.
+ *  - Quantizer groups are `group` consecutive columns of a row of the rotated
+ *    matrix. Lloyd-Max: s = sqrt(mean(x^2)) over the group; code = number of
+ *    fp32 midpoints t_k (of neighbouring fp32 centroids) with x/s > t_k.
+ *    Absmax: s = max|x| / (2^(b-1) - 1); code = clamp(rint(x/s), -qmax, qmax)
+ *    + 2^(b-1), so 4-bit codes are 1..15. Scales are stored as IEEE fp16
+ *    (round to nearest even, saturating at 65504) and codes are computed
+ *    with the stored scale. A group whose stored scale is 0 gets the middle
+ *    code (2^(b-1)) and dequantizes to 0.
+ *  - Packing: code i of a row occupies bits [b*i, b*i + b) of that row's
+ *    little-endian bitstream (first code in the low bits of byte 0); rows of
+ *    `codes` are cols*b/8 bytes apart. Scales are a separate [rows x
+ *    cols/group] fp16 array.
+ *
+ * Memory and errors:
+ *  - All tensor pointers passed to compute calls are DEVICE pointers owned by
+ *    the caller (e.g. torch tensors) unless a parameter says "host". Compute
+ *    calls are asynchronous on the given CUDA stream (NULL = legacy default
+ *    stream) and never synchronise; the library allocates no device memory
+ *    after plan creation.
+ *  - Every call returns a harp_status (0 = HARP_OK). Arguments are checked on
+ *    the host before any launch; a rejected call launches nothing and leaves
+ *    outputs untouched. A compute call on an empty matrix (rows or cols 0)
+ *    checks its plan, codebook and shapes, then returns HARP_OK without
+ *    touching any pointer. Kernels never trap or assert. HARP_ERR_CUDA reports a
+ *    launch error (cudaGetLastError after the launch); asynchronous execution
+ *    errors surface at the caller's next synchronisation.
+ *  - There is no CPU fallback: without a CUDA device, plan creation returns
+ *    HARP_ERR_CUDA.
+ */
+#ifndef HARP_H_
+#define HARP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum harp_status {
+    HARP_OK = 0,
+    HARP_ERR_INVALID_ARG = 1,   /* NULL where a pointer is required, bad enum value */
+    HARP_ERR_SHAPE = 2,         /* prod b_t != d, d != rows/cols, group does not divide cols, ... */
+    HARP_ERR_UNSUPPORTED = 3,   /* radix outside [1, 64], more than 16 stages, bits not in {2,3,4} */
+    HARP_ERR_ALIGNMENT = 4,     /* device pointer or leading dimension not aligned (see each call) */
+    HARP_ERR_WORKSPACE = 5,     /* workspace NULL or smaller than harp_workspace_size() */
+    HARP_ERR_CUDA = 6,          /* CUDA runtime error (no device, launch failure) */
+    HARP_ERR_ALLOC = 7          /* host or device allocation failed at plan / codebook creation */
+} harp_status;
+
+enum harp_dtype { HARP_F32 = 0, HARP_BF16 = 1 };
+enum harp_side { HARP_RIGHT = 0, HARP_LEFT = 1 };
+enum harp_dir { HARP_FWD = 0, HARP_INV = 1 };
+enum harp_quant_kind { HARP_LLOYD_MAX = 0, HARP_ABSMAX = 1 };
+enum harp_block_kind { HARP_BLOCKS_HADAMARD = 0, HARP_BLOCKS_QR = 1, HARP_BLOCKS_CAYLEY = 2 };
+
+#define HARP_MAX_STAGES 16
+#define HARP_MAX_RADIX 64
+
+typedef struct harp_plan_s *harp_plan_t;
+typedef struct harp_codebook_s *harp_codebook_t;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *harp_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int harp_version(void);
+
+/* --------------------------------------------------------------- plan objects */
+
+/* Create a processor plan on the current CUDA device  [HARP 2.1, 2.2].
+ *  d      vector length the processor acts on (cols for HARP_RIGHT, rows for
+ *         HARP_LEFT), 1 <= d <= 2^31 - 1.
+ *  m      number of stages, 1 <= m <= HARP_MAX_STAGES.
+ *  radix  host [m]; each b_t in [1, HARP_MAX_RADIX]; prod b_t must equal d.
+ *  blocks host [m] pointers; blocks[t] points to d/b_t row-major b_t x b_t
+ *         float blocks (block c at offset c*b_t*b_t, entry [k][j] = output
+ *         k, input j). The blocks are used as given; forward and inverse are
+ *         exact inverses only if they are orthogonal.
+ *  signs  host [d] of +1/-1 (any float is accepted and multiplied in), or
+ *         NULL for all +1.
+ * The plan copies blocks and signs to device memory (synchronously) and owns
+ * that copy until harp_plan_destroy. Errors: INVALID_ARG (NULL out/radix/
+ * blocks), UNSUPPORTED, SHAPE, CUDA, ALLOC. */
+int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
+                     const float *const *blocks, const float *signs);
+
+/* Release a plan and its device memory. NULL is accepted. The caller must
+ * ensure no launch that uses the plan is still running. */
+int harp_plan_destroy(harp_plan_t plan);
+
+/* Read back a plan's shape: d, m and radix (host [HARP_MAX_STAGES]); any
+ * output pointer may be NULL. */
+int harp_plan_info(harp_plan_t plan, int64_t *d, int *m, int32_t *radix);
+
+/* Build one stage's blocks from raw Gaussian draws, on the host, in double
+ * precision, rounded to float  [HARP 2.1, 2.2]:
+ *  HARP_BLOCKS_HADAMARD  every group gets the base mixer G_b: the normalised
+ *                        Sylvester Hadamard if b is a power of two, else the
+ *                        Q factor (positive R diagonal) of `base_gauss`.
+ *  HARP_BLOCKS_QR        group c gets the Q factor (positive R diagonal) of
+ *                        gauss[c] (a random orthogonal block).
+ *  HARP_BLOCKS_CAYLEY    group c gets Q_c G_b, with Q_c the Cayley map
+ *                        (I - A)^-1 (I + A) of A = skew_scale * S_c, S_c the
+ *                        skew-symmetric matrix whose strict upper triangle is
+ *                        gauss[c]'s; for b = 2, Q_c is the Givens rotation
+ *                        [[cos a, -sin a], [sin a, cos a]], a =
+ *                        skew_scale * gauss[c][0][1]. skew_scale = 0 gives
+ *                        back G_b exactly.
+ *  gauss      host [n_groups][b][b] doubles (ignored for HADAMARD), row-major.
+ *  base_gauss host [b][b] doubles, needed only when b is not a power of two
+ *             and kind != QR.
+ *  out        host [n_groups][b][b] floats.
+ * Errors: INVALID_ARG, UNSUPPORTED (b outside [1, 64]), SHAPE (singular
+ * input). */
+int harp_stage_blocks(int kind, int b, int64_t n_groups, const double *gauss,
+                      const double *base_gauss, double skew_scale, float *out);
+
+/* Lloyd-Max centroids for N(0,1) with 2^bits levels  [PolarQuant 2], computed
+ * on the host (double precision, rounded to float): ascending, odd-symmetric.
+ * out: host [2^bits]. bits in {2, 3, 4}. */
+int harp_lloyd_max_centroids(int bits, float *out);
+
+/* Create a quantizer description  [PolarQuant 1, 2].
+ *  kind       HARP_LLOYD_MAX or HARP_ABSMAX.
+ *  bits       2, 3 or 4.
+ *  group      elements per scale group along a row: a positive multiple of
+ *             32 (UNSUPPORTED otherwise); must divide cols at each call
+ *             (group = cols gives one scale per row).
+ *  centroids  host [2^bits] ascending floats for HARP_LLOYD_MAX, or NULL for
+ *             the built-in N(0,1) Lloyd-Max table; ignored for absmax.
+ * Host-only object (no device memory); the tables travel as kernel arguments.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALLOC. */
+int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group,
+                         const float *centroids);
+int harp_codebook_destroy(harp_codebook_t cb);
+
+/* Copy a codebook's fp32 tables to host memory: centroids [2^bits] (absmax:
+ * the integer levels code - 2^(b-1)) and thresholds [2^bits - 1]; either may
+ * be NULL. */
+int harp_codebook_tables(harp_codebook_t cb, float *centroids, float *thresholds);
+
+/* Bytes of device workspace the fused two-sided calls need for a
+ * [rows x cols] matrix: rows*cols*4 (an fp32 intermediate) when `left` is
+ * not NULL, else 0. */
+int harp_workspace_size(harp_plan_t left, harp_plan_t right, int64_t rows, int64_t cols,
+                        size_t *bytes);
+
+/* ------------------------------------------------------------ compute calls */
+
+/* Apply a processor to the rows (HARP_RIGHT, plan d = cols) or the columns
+ * (HARP_LEFT, plan d = rows) of a row-major matrix, forward (M) or inverse
+ * (M^T)  [HARP 2.1; 5].
+ *  in, out      device; element [r][c] at r*ld + c; in_dtype / out_dtype are
+ *               HARP_F32 or HARP_BF16 (bf16 output rounds to nearest even).
+ *               in and out must not overlap.
+ *  ld_in/ld_out leading dimensions in elements, >= cols, multiples of 4.
+ *  Alignment: in and out 16-byte aligned.
+ * Arithmetic is fp32 with fp32 blocks. */
+int harp_rotate(harp_plan_t plan, int side, int dir, const void *in, int in_dtype,
+                void *out, int out_dtype, int64_t rows, int64_t cols, int64_t ld_in,
+                int64_t ld_out, void *stream);
+
+/* Group-wise quantize an (already rotated) row-major matrix  [PolarQuant 2].
+ *  in      device [rows x cols], leading dimension ld_in (multiple of 4).
+ *  codes   device [rows x cols*bits/8] bytes (cols*bits % 8 == 0; packed as
+ *          described above); scales device [rows x cols/group] fp16 bits.
+ *  Alignment: in 16 bytes, codes 4 bytes, scales 2 bytes. */
+int harp_quantize(harp_codebook_t cb, const void *in, int in_dtype, int64_t rows,
+                  int64_t cols, int64_t ld_in, uint8_t *codes, uint16_t *scales,
+                  void *stream);
+
+/* Inverse of harp_quantize: out[r][c] = s * centroid[code] (Lloyd-Max) or
+ * s * (code - 2^(b-1)) (absmax)  [PolarQuant 2]. out: device, ld_out >= cols,
+ * multiple of 4, 16-byte aligned. */
+int harp_dequantize(harp_codebook_t cb, const uint8_t *codes, const uint16_t *scales,
+                    int64_t rows, int64_t cols, void *out, int out_dtype, int64_t ld_out,
+                    void *stream);
+
+/* Fused forward path: W' = M_L W M_R^T (left may be NULL for right-only),
+ * then group-wise quantize and pack W'  [HARP 2.1, 3; PolarQuant 2].
+ *  in           device [rows x cols], contiguous (ld = cols), F32 or BF16.
+ *  codes/scales as in harp_quantize.
+ *  rotated_out  optional device fp32 [rows x cols] copy of W' (NULL = none).
+ *  workspace    device, >= harp_workspace_size bytes, 16-byte aligned
+ *               (may be NULL when the size is 0).
+ * right->d must equal cols and left->d rows. */
+int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,
+                         const void *in, int in_dtype, int64_t rows, int64_t cols,
+                         uint8_t *codes, uint16_t *scales, float *rotated_out,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/* Fused inverse path: dequantize, then W = M_L^T W' M_R  [HARP 5;
+ * PolarQuant 2]. out: device [rows x cols] contiguous, F32 or BF16.
+ * Workspace as for harp_rotate_quantize. */
+int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,
+                             const uint8_t *codes, const uint16_t *scales, int64_t rows,
+                             int64_t cols, void *out, int out_dtype, void *workspace,
+                             size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HARP_H_ */

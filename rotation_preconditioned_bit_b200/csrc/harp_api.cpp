@@ -1,0 +1,563 @@
+// harp_api.cpp -- the C ABI of libharp (declared in include/harp.h): argument
+// checking, plan and codebook objects, host-side block and codebook
+// construction, and the launch sequences of the fused paths.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <limits>
+#include <new>
+#include <vector>
+
+#include "harp.h"
+#include "harp_internal.h"
+
+struct harp_plan_s {
+    int device;
+    int64_t d;
+    int m;
+    int32_t radix[HARP_MAX_STAGES];
+    void *mem;  // one device allocation: signs, then each stage's fwd and inv blocks
+    harp::PlanDev dev;
+};
+
+struct harp_codebook_s {
+    harp::QuantDev q;
+    int K;
+};
+
+namespace {
+
+constexpr size_t kMaxTileBytes = 232448;
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(int err) { return err == 0 ? HARP_OK : HARP_ERR_CUDA; }
+
+// ------------------------------------------------------------ block makers
+// HARP (gist.science paper 2605.29843) section 2.2: B = Q(theta) G_b.
+
+// Normalised Sylvester Hadamard, entry (-1)^popcount(i & j) / sqrt(b).
+void sylvester(int b, std::vector<double> &H) {
+    H.assign(static_cast<size_t>(b) * b, 0.0);
+    const double sc = 1.0 / std::sqrt(static_cast<double>(b));
+    for (int i = 0; i < b; ++i)
+        for (int j = 0; j < b; ++j)
+            H[static_cast<size_t>(i) * b + j] = (__builtin_popcount(static_cast<unsigned>(i & j)) & 1) ? -sc : sc;
+}
+
+// Q of G = Q R with diag(R) > 0, by Householder reflections.
+bool householder_q(int b, const double *G, std::vector<double> &Q) {
+    std::vector<double> R(G, G + static_cast<size_t>(b) * b);
+    std::vector<double> V(static_cast<size_t>(b) * b, 0.0);  // reflector k in row k
+    std::vector<double> beta(b, 0.0);
+    for (int k = 0; k < b; ++k) {
+        double nrm = 0.0;
+        for (int i = k; i < b; ++i) nrm += R[static_cast<size_t>(i) * b + k] * R[static_cast<size_t>(i) * b + k];
+        nrm = std::sqrt(nrm);
+        if (nrm == 0.0) return false;
+        const double x0 = R[static_cast<size_t>(k) * b + k];
+        const double alpha = (x0 >= 0.0) ? -nrm : nrm;
+        double vn = 0.0;
+        for (int i = k; i < b; ++i) {
+            double v = R[static_cast<size_t>(i) * b + k] - (i == k ? alpha : 0.0);
+            V[static_cast<size_t>(k) * b + i] = v;
+            vn += v * v;
+        }
+        beta[k] = (vn > 0.0) ? 2.0 / vn : 0.0;
+        for (int j = k; j < b; ++j) {           // R <- (I - beta v v^T) R
+            double dot = 0.0;
+            for (int i = k; i < b; ++i) dot += V[static_cast<size_t>(k) * b + i] * R[static_cast<size_t>(i) * b + j];
+            dot *= beta[k];
+            for (int i = k; i < b; ++i) R[static_cast<size_t>(i) * b + j] -= dot * V[static_cast<size_t>(k) * b + i];
+        }
+    }
+    // Q = H_0 H_1 ... H_{b-1}: apply the reflectors to I in reverse order
+    Q.assign(static_cast<size_t>(b) * b, 0.0);
+    for (int i = 0; i < b; ++i) Q[static_cast<size_t>(i) * b + i] = 1.0;
+    for (int k = b - 1; k >= 0; --k)
+        for (int j = 0; j < b; ++j) {
+            double dot = 0.0;
+            for (int i = k; i < b; ++i) dot += V[static_cast<size_t>(k) * b + i] * Q[static_cast<size_t>(i) * b + j];
+            dot *= beta[k];
+            for (int i = k; i < b; ++i) Q[static_cast<size_t>(i) * b + j] -= dot * V[static_cast<size_t>(k) * b + i];
+        }
+    // make diag(R) positive: flip column k of Q where R[k][k] < 0
+    for (int k = 0; k < b; ++k)
+        if (R[static_cast<size_t>(k) * b + k] < 0.0)
+            for (int i = 0; i < b; ++i) Q[static_cast<size_t>(i) * b + k] = -Q[static_cast<size_t>(i) * b + k];
+    return true;
+}
+
+// Cayley map (I - A)^-1 (I + A) by Gauss-Jordan elimination with pivoting.
+bool cayley(int b, const std::vector<double> &A, std::vector<double> &Q) {
+    const int w = 2 * b;
+    std::vector<double> M(static_cast<size_t>(b) * w);
+    for (int i = 0; i < b; ++i)
+        for (int j = 0; j < b; ++j) {
+            const double id = (i == j) ? 1.0 : 0.0;
+            M[static_cast<size_t>(i) * w + j] = id - A[static_cast<size_t>(i) * b + j];
+            M[static_cast<size_t>(i) * w + b + j] = id + A[static_cast<size_t>(i) * b + j];
+        }
+    for (int c = 0; c < b; ++c) {
+        int p = c;
+        for (int r = c + 1; r < b; ++r)
+            if (std::fabs(M[static_cast<size_t>(r) * w + c]) > std::fabs(M[static_cast<size_t>(p) * w + c])) p = r;
+        if (M[static_cast<size_t>(p) * w + c] == 0.0) return false;
+        if (p != c)
+            for (int j = 0; j < w; ++j) std::swap(M[static_cast<size_t>(p) * w + j], M[static_cast<size_t>(c) * w + j]);
+        const double inv = 1.0 / M[static_cast<size_t>(c) * w + c];
+        for (int j = 0; j < w; ++j) M[static_cast<size_t>(c) * w + j] *= inv;
+        for (int r = 0; r < b; ++r) {
+            if (r == c) continue;
+            const double f = M[static_cast<size_t>(r) * w + c];
+            if (f == 0.0) continue;
+            for (int j = 0; j < w; ++j) M[static_cast<size_t>(r) * w + j] -= f * M[static_cast<size_t>(c) * w + j];
+        }
+    }
+    Q.assign(static_cast<size_t>(b) * b, 0.0);
+    for (int i = 0; i < b; ++i)
+        for (int j = 0; j < b; ++j) Q[static_cast<size_t>(i) * b + j] = M[static_cast<size_t>(i) * w + b + j];
+    return true;
+}
+
+// ------------------------------------------------------------ Lloyd-Max
+// PolarQuant (gist.science paper 2603.29078) section 2: MSE-optimal scalar
+// codebook for N(0,1). Solved on the positive half (the optimum is odd-
+// symmetric and, for even K, has a threshold at 0): each centroid is its
+// cell's conditional mean and each inner threshold the midpoint of its two
+// centroids; iterate from evenly spaced levels until nothing moves.
+double npdf(double z) { return std::exp(-0.5 * z * z) * 0.39894228040143267794; }
+
+// P(a < Z < b) for 0 <= a < b, from the upper tail to keep precision.
+double nmass(double a, double b) {
+    const double ta = 0.5 * std::erfc(a * 0.70710678118654752440);
+    const double tb = std::isinf(b) ? 0.0 : 0.5 * std::erfc(b * 0.70710678118654752440);
+    return ta - tb;
+}
+
+bool lloyd_max_half(int K, std::vector<double> &pos) {
+    const int n = K / 2;
+    pos.resize(n);
+    for (int k = 0; k < n; ++k) pos[k] = (k + 0.5) * (3.0 / n);
+    std::vector<double> t(n + 1);
+    for (int it = 0; it < 1000000; ++it) {
+        t[0] = 0.0;
+        for (int k = 1; k < n; ++k) t[k] = 0.5 * (pos[k - 1] + pos[k]);
+        t[n] = std::numeric_limits<double>::infinity();
+        double moved = 0.0;
+        for (int k = 0; k < n; ++k) {
+            const double hi = std::isinf(t[k + 1]) ? 0.0 : npdf(t[k + 1]);
+            const double c = (npdf(t[k]) - hi) / nmass(t[k], t[k + 1]);
+            moved = std::fmax(moved, std::fabs(c - pos[k]));
+            pos[k] = c;
+        }
+        if (moved <= 1e-15) return true;
+    }
+    return true;
+}
+
+}  // namespace
+
+// ================================================================ C ABI
+
+extern "C" {
+
+const char *harp_status_string(int status) {
+    switch (status) {
+        case HARP_OK: return "ok";
+        case HARP_ERR_INVALID_ARG: return "invalid argument";
+        case HARP_ERR_SHAPE: return "shape mismatch";
+        case HARP_ERR_UNSUPPORTED: return "unsupported configuration";
+        case HARP_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+        case HARP_ERR_WORKSPACE: return "workspace missing or too small";
+        case HARP_ERR_CUDA: return "CUDA error";
+        case HARP_ERR_ALLOC: return "allocation failed";
+        default: return "unknown status";
+    }
+}
+
+int harp_version(void) { return 100; }
+
+int harp_stage_blocks(int kind, int b, int64_t n_groups, const double *gauss,
+                      const double *base_gauss, double skew_scale, float *out) {
+    if (!out || n_groups < 0) return HARP_ERR_INVALID_ARG;
+    if (b < 1 || b > HARP_MAX_RADIX) return HARP_ERR_UNSUPPORTED;
+    if (kind != HARP_BLOCKS_HADAMARD && kind != HARP_BLOCKS_QR && kind != HARP_BLOCKS_CAYLEY)
+        return HARP_ERR_INVALID_ARG;
+    if (kind != HARP_BLOCKS_HADAMARD && !gauss && n_groups > 0) return HARP_ERR_INVALID_ARG;
+    const bool pow2 = (b & (b - 1)) == 0;
+    std::vector<double> G;
+    if (kind != HARP_BLOCKS_QR) {
+        if (pow2) {
+            sylvester(b, G);
+        } else {
+            if (!base_gauss) return HARP_ERR_INVALID_ARG;
+            if (!householder_q(b, base_gauss, G)) return HARP_ERR_SHAPE;
+        }
+    }
+    const size_t bb = static_cast<size_t>(b) * b;
+    std::vector<double> Q, A(bb), B(bb);
+    for (int64_t c = 0; c < n_groups; ++c) {
+        const double *g = gauss ? gauss + c * bb : nullptr;
+        if (kind == HARP_BLOCKS_HADAMARD) {
+            B = G;
+        } else if (kind == HARP_BLOCKS_QR) {
+            if (!householder_q(b, g, B)) return HARP_ERR_SHAPE;
+        } else {
+            if (b == 2) {
+                const double a = skew_scale * g[1];
+                Q = {std::cos(a), -std::sin(a), std::sin(a), std::cos(a)};
+            } else {
+                for (int i = 0; i < b; ++i)
+                    for (int j = 0; j < b; ++j)
+                        A[static_cast<size_t>(i) * b + j] =
+                            (i < j) ? skew_scale * g[static_cast<size_t>(i) * b + j]
+                          : (i > j) ? -skew_scale * g[static_cast<size_t>(j) * b + i] : 0.0;
+                if (!cayley(b, A, Q)) return HARP_ERR_SHAPE;
+            }
+            for (int i = 0; i < b; ++i)
+                for (int j = 0; j < b; ++j) {
+                    double acc = 0.0;
+                    for (int k = 0; k < b; ++k) acc += Q[static_cast<size_t>(i) * b + k] * G[static_cast<size_t>(k) * b + j];
+                    B[static_cast<size_t>(i) * b + j] = acc;
+                }
+        }
+        for (size_t e = 0; e < bb; ++e) out[c * bb + e] = static_cast<float>(B[e]);
+    }
+    return HARP_OK;
+}
+
+int harp_lloyd_max_centroids(int bits, float *out) {
+    if (!out) return HARP_ERR_INVALID_ARG;
+    if (bits < 2 || bits > 4) return HARP_ERR_UNSUPPORTED;
+    const int K = 1 << bits;
+    std::vector<double> pos;
+    lloyd_max_half(K, pos);
+    for (int k = 0; k < K / 2; ++k) {
+        out[K / 2 + k] = static_cast<float>(pos[k]);
+        out[K / 2 - 1 - k] = static_cast<float>(-pos[k]);
+    }
+    return HARP_OK;
+}
+
+int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
+                     const float *const *blocks, const float *signs) {
+    if (!out || !radix || !blocks) return HARP_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (m < 1 || m > HARP_MAX_STAGES) return HARP_ERR_UNSUPPORTED;
+    if (d < 1 || d > std::numeric_limits<int32_t>::max()) return HARP_ERR_SHAPE;
+    int64_t prod = 1;
+    for (int t = 0; t < m; ++t) {
+        if (radix[t] < 1 || radix[t] > HARP_MAX_RADIX) return HARP_ERR_UNSUPPORTED;
+        if (!blocks[t]) return HARP_ERR_INVALID_ARG;
+        prod *= radix[t];
+        if (prod > d) return HARP_ERR_SHAPE;
+    }
+    if (prod != d) return HARP_ERR_SHAPE;
+    if (static_cast<size_t>(d) * 4 > kMaxTileBytes) return HARP_ERR_UNSUPPORTED;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HARP_ERR_CUDA; }
+
+    // host staging of the device layout
+    const size_t sign_floats = (static_cast<size_t>(d) + 3) & ~static_cast<size_t>(3);
+    size_t total = sign_floats;
+    std::vector<size_t> off(m);
+    for (int t = 0; t < m; ++t) {
+        const int kpad = (radix[t] + 3) & ~3;
+        off[t] = total;
+        total += 2 * static_cast<size_t>(d) * kpad;   // fwd then inv
+    }
+    std::vector<float> host;
+    try { host.assign(total, 0.0f); } catch (...) { return HARP_ERR_ALLOC; }
+    for (int64_t i = 0; i < d; ++i) host[i] = signs ? signs[i] : 1.0f;
+    for (int t = 0; t < m; ++t) {
+        const int b = radix[t], kpad = (b + 3) & ~3;
+        const int64_t ng = d / b;
+        float *fwd = host.data() + off[t];
+        float *inv = fwd + static_cast<size_t>(d) * kpad;
+        for (int64_t c = 0; c < ng; ++c) {
+            const float *B = blocks[t] + c * b * b;
+            for (int k = 0; k < b; ++k)
+                for (int j = 0; j < b; ++j) {
+                    fwd[(c * b + j) * kpad + k] = B[k * b + j];
+                    inv[(c * b + k) * kpad + j] = B[k * b + j];
+                }
+        }
+    }
+    harp_plan_s *p = new (std::nothrow) harp_plan_s();
+    if (!p) return HARP_ERR_ALLOC;
+    if (cudaMalloc(&p->mem, total * sizeof(float)) != cudaSuccess) {
+        cudaGetLastError();
+        delete p;
+        return HARP_ERR_ALLOC;
+    }
+    if (cudaMemcpy(p->mem, host.data(), total * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(p->mem);
+        delete p;
+        return HARP_ERR_CUDA;
+    }
+    p->device = dev;
+    p->d = d;
+    p->m = m;
+    for (int t = 0; t < HARP_MAX_STAGES; ++t) p->radix[t] = (t < m) ? radix[t] : 0;
+    float *base = static_cast<float *>(p->mem);
+    p->dev.d = d;
+    p->dev.m = m;
+    p->dev.signs = base;
+    int64_t s = d;
+    for (int t = 0; t < m; ++t) {
+        const int b = radix[t], kpad = (b + 3) & ~3;
+        s /= b;
+        p->dev.st[t].b = b;
+        p->dev.st[t].kpad = kpad;
+        p->dev.st[t].s = s;
+        p->dev.st[t].fwd = base + off[t];
+        p->dev.st[t].inv = base + off[t] + static_cast<size_t>(d) * kpad;
+    }
+    *out = p;
+    return HARP_OK;
+}
+
+int harp_plan_destroy(harp_plan_t plan) {
+    if (!plan) return HARP_OK;
+    int st = HARP_OK;
+    if (plan->mem && cudaFree(plan->mem) != cudaSuccess) { cudaGetLastError(); st = HARP_ERR_CUDA; }
+    delete plan;
+    return st;
+}
+
+int harp_plan_info(harp_plan_t plan, int64_t *d, int *m, int32_t *radix) {
+    if (!plan) return HARP_ERR_INVALID_ARG;
+    if (d) *d = plan->d;
+    if (m) *m = plan->m;
+    if (radix) std::memcpy(radix, plan->radix, sizeof(plan->radix));
+    return HARP_OK;
+}
+
+int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group,
+                         const float *centroids) {
+    if (!out) return HARP_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (kind != HARP_LLOYD_MAX && kind != HARP_ABSMAX) return HARP_ERR_INVALID_ARG;
+    if (bits < 2 || bits > 4) return HARP_ERR_UNSUPPORTED;
+    if (group <= 0) return HARP_ERR_SHAPE;
+    if (group % 32 != 0 || group > std::numeric_limits<int32_t>::max()) return HARP_ERR_UNSUPPORTED;
+    harp_codebook_s *cb = new (std::nothrow) harp_codebook_s();
+    if (!cb) return HARP_ERR_ALLOC;
+    const int K = 1 << bits;
+    cb->K = K;
+    cb->q.kind = kind;
+    cb->q.bits = bits;
+    cb->q.group = static_cast<int>(group);
+    if (kind == HARP_LLOYD_MAX) {
+        float c[16];
+        if (centroids) {
+            for (int k = 0; k < K; ++k) c[k] = centroids[k];
+            for (int k = 0; k + 1 < K; ++k)
+                if (!(c[k] < c[k + 1])) { delete cb; return HARP_ERR_INVALID_ARG; }
+        } else {
+            harp_lloyd_max_centroids(bits, c);
+        }
+        for (int k = 0; k < K; ++k) cb->q.level[k] = c[k];
+        for (int k = 0; k + 1 < K; ++k)
+            cb->q.thr[k] = static_cast<float>(0.5 * (static_cast<double>(c[k]) + static_cast<double>(c[k + 1])));
+    } else {
+        for (int k = 0; k < K; ++k) cb->q.level[k] = static_cast<float>(k - K / 2);
+    }
+    *out = cb;
+    return HARP_OK;
+}
+
+int harp_codebook_destroy(harp_codebook_t cb) {
+    delete cb;
+    return HARP_OK;
+}
+
+int harp_codebook_tables(harp_codebook_t cb, float *centroids, float *thresholds) {
+    if (!cb) return HARP_ERR_INVALID_ARG;
+    if (centroids) for (int k = 0; k < cb->K; ++k) centroids[k] = cb->q.level[k];
+    if (thresholds) for (int k = 0; k + 1 < cb->K; ++k) thresholds[k] = cb->q.thr[k];
+    return HARP_OK;
+}
+
+int harp_workspace_size(harp_plan_t left, harp_plan_t right, int64_t rows, int64_t cols,
+                        size_t *bytes) {
+    (void)right;
+    if (!bytes || rows < 0 || cols < 0) return HARP_ERR_INVALID_ARG;
+    *bytes = left ? static_cast<size_t>(rows) * static_cast<size_t>(cols) * 4 : 0;
+    return HARP_OK;
+}
+
+static bool valid_dtype(int t) { return t == HARP_F32 || t == HARP_BF16; }
+static size_t dtype_size(int t) { return t == HARP_F32 ? 4 : 2; }
+
+int harp_rotate(harp_plan_t plan, int side, int dir, const void *in, int in_dtype, void *out,
+                int out_dtype, int64_t rows, int64_t cols, int64_t ld_in, int64_t ld_out,
+                void *stream) {
+    if (!plan) return HARP_ERR_INVALID_ARG;
+    if (side != HARP_RIGHT && side != HARP_LEFT) return HARP_ERR_INVALID_ARG;
+    if (dir != HARP_FWD && dir != HARP_INV) return HARP_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return HARP_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0) return HARP_ERR_SHAPE;
+    if ((side == HARP_RIGHT ? cols : rows) != plan->d) return HARP_ERR_SHAPE;
+    if (ld_in < cols || ld_out < cols) return HARP_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!in || !out) return HARP_ERR_INVALID_ARG;
+    if (ld_in % 4 || ld_out % 4 || !aligned(in, 16) || !aligned(out, 16)) return HARP_ERR_ALIGNMENT;
+    const char *ib = static_cast<const char *>(in);
+    const char *ob = static_cast<const char *>(out);
+    const size_t in_bytes = rows ? (static_cast<size_t>(rows - 1) * ld_in + cols) * dtype_size(in_dtype) : 0;
+    const size_t out_bytes = rows ? (static_cast<size_t>(rows - 1) * ld_out + cols) * dtype_size(out_dtype) : 0;
+    if (ib < ob + out_bytes && ob < ib + in_bytes) return HARP_ERR_INVALID_ARG;
+    harp::VecLaunch L{};
+    L.side = side;
+    L.dir = dir;
+    L.pro = (in_dtype == HARP_F32) ? harp::PRO_F32 : harp::PRO_BF16;
+    L.epi = (out_dtype == HARP_F32) ? harp::EPI_F32 : harp::EPI_BF16;
+    L.nvec = (side == HARP_RIGHT) ? rows : cols;
+    L.in = in;
+    L.ld_in = ld_in;
+    L.out = out;
+    L.ld_out = ld_out;
+    return cuda_status(harp::launch_vec(plan->dev, nullptr, L, stream));
+}
+
+static int check_codec(harp_codebook_t cb, int64_t rows, int64_t cols) {
+    if (!cb) return HARP_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0) return HARP_ERR_SHAPE;
+    if (cols % cb->q.group) return HARP_ERR_SHAPE;
+    return HARP_OK;
+}
+
+int harp_quantize(harp_codebook_t cb, const void *in, int in_dtype, int64_t rows, int64_t cols,
+                  int64_t ld_in, uint8_t *codes, uint16_t *scales, void *stream) {
+    int st = check_codec(cb, rows, cols);
+    if (st) return st;
+    if (!valid_dtype(in_dtype)) return HARP_ERR_INVALID_ARG;
+    if (ld_in < cols) return HARP_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!in || !codes || !scales) return HARP_ERR_INVALID_ARG;
+    if (ld_in % 4 || !aligned(in, 16) || !aligned(codes, 4) || !aligned(scales, 2)) return HARP_ERR_ALIGNMENT;
+    return cuda_status(harp::launch_quantize(cb->q, in, in_dtype, rows, cols, ld_in, codes, scales, stream));
+}
+
+int harp_dequantize(harp_codebook_t cb, const uint8_t *codes, const uint16_t *scales, int64_t rows,
+                    int64_t cols, void *out, int out_dtype, int64_t ld_out, void *stream) {
+    int st = check_codec(cb, rows, cols);
+    if (st) return st;
+    if (!valid_dtype(out_dtype)) return HARP_ERR_INVALID_ARG;
+    if (ld_out < cols) return HARP_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
+    if (ld_out % 4 || !aligned(out, 16) || !aligned(scales, 2)) return HARP_ERR_ALIGNMENT;
+    return cuda_status(harp::launch_dequantize(cb->q, codes, scales, rows, cols, out, out_dtype, ld_out, stream));
+}
+
+static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int64_t rows,
+                      int64_t cols, void *workspace, size_t ws_bytes) {
+    if (!right || !cb) return HARP_ERR_INVALID_ARG;
+    int st = check_codec(cb, rows, cols);
+    if (st) return st;
+    if (right->d != cols) return HARP_ERR_SHAPE;
+    if (left && left->d != rows) return HARP_ERR_SHAPE;
+    if (harp::vec_tile(cols, harp::EPI_QUANT, cb->q.group) == 0) return HARP_ERR_UNSUPPORTED;
+    if (left) {
+        const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(cols) * 4;
+        if (need && (!workspace || ws_bytes < need)) return HARP_ERR_WORKSPACE;
+        if (workspace && !aligned(workspace, 16)) return HARP_ERR_ALIGNMENT;
+    }
+    return HARP_OK;
+}
+
+int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, const void *in,
+                         int in_dtype, int64_t rows, int64_t cols, uint8_t *codes,
+                         uint16_t *scales, float *rotated_out, void *workspace, size_t ws_bytes,
+                         void *stream) {
+    int st = check_pair(left, right, cb, rows, cols, workspace, ws_bytes);
+    if (st) return st;
+    if (!valid_dtype(in_dtype)) return HARP_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!in || !codes || !scales) return HARP_ERR_INVALID_ARG;
+    if (!aligned(in, 16) || !aligned(codes, 4) || !aligned(scales, 2) ||
+        (rotated_out && !aligned(rotated_out, 16)) || cols % 4)
+        return HARP_ERR_ALIGNMENT;
+    const int pro_in = (in_dtype == HARP_F32) ? harp::PRO_F32 : harp::PRO_BF16;
+    const void *row_in = in;
+    int row_pro = pro_in;
+    if (left) {
+        harp::VecLaunch Lc{};
+        Lc.side = HARP_LEFT;
+        Lc.dir = HARP_FWD;
+        Lc.pro = pro_in;
+        Lc.epi = harp::EPI_F32;
+        Lc.nvec = cols;
+        Lc.in = in;
+        Lc.ld_in = cols;
+        Lc.out = workspace;
+        Lc.ld_out = cols;
+        st = cuda_status(harp::launch_vec(left->dev, nullptr, Lc, stream));
+        if (st) return st;
+        row_in = workspace;
+        row_pro = harp::PRO_F32;
+    }
+    harp::VecLaunch Lr{};
+    Lr.side = HARP_RIGHT;
+    Lr.dir = HARP_FWD;
+    Lr.pro = row_pro;
+    Lr.epi = rotated_out ? harp::EPI_QUANT_F32 : harp::EPI_QUANT;
+    Lr.nvec = rows;
+    Lr.in = row_in;
+    Lr.ld_in = cols;
+    Lr.out = rotated_out;
+    Lr.ld_out = cols;
+    Lr.codes = codes;
+    Lr.scales = scales;
+    return cuda_status(harp::launch_vec(right->dev, &cb->q, Lr, stream));
+}
+
+int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,
+                             const uint8_t *codes, const uint16_t *scales, int64_t rows,
+                             int64_t cols, void *out, int out_dtype, void *workspace,
+                             size_t ws_bytes, void *stream) {
+    int st = check_pair(left, right, cb, rows, cols, workspace, ws_bytes);
+    if (st) return st;
+    if (!valid_dtype(out_dtype)) return HARP_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(scales, 2) || cols % 4) return HARP_ERR_ALIGNMENT;
+    harp::VecLaunch Lr{};
+    Lr.side = HARP_RIGHT;
+    Lr.dir = HARP_INV;
+    Lr.pro = harp::PRO_CODES;
+    Lr.nvec = rows;
+    Lr.in_codes = codes;
+    Lr.in_scales = scales;
+    Lr.ld_out = cols;
+    if (left) {
+        Lr.epi = harp::EPI_F32;
+        Lr.out = workspace;
+    } else {
+        Lr.epi = (out_dtype == HARP_F32) ? harp::EPI_F32 : harp::EPI_BF16;
+        Lr.out = out;
+    }
+    st = cuda_status(harp::launch_vec(right->dev, &cb->q, Lr, stream));
+    if (st || !left) return st;
+    harp::VecLaunch Lc{};
+    Lc.side = HARP_LEFT;
+    Lc.dir = HARP_INV;
+    Lc.pro = harp::PRO_F32;
+    Lc.epi = (out_dtype == HARP_F32) ? harp::EPI_F32 : harp::EPI_BF16;
+    Lc.nvec = cols;
+    Lc.in = workspace;
+    Lc.ld_in = cols;
+    Lc.out = out;
+    Lc.ld_out = cols;
+    return cuda_status(harp::launch_vec(left->dev, nullptr, Lc, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Internal interface between the C ABI (harp_api.cpp) and the kernels
+// (harp_kernels.cu). Not installed; the public surface is include/harp.h.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "harp.h"
+
+namespace harp {
+
+// One stride stage as the kernels see it. Blocks are stored twice, padded
+// along the output index to a multiple of 4 so a lane reads four outputs'
+// coefficients with one 16-byte load:
+//   fwd[c][j][k] = B_{t,c}[k][j]   (forward: out k, in j)
+//   inv[c][k][j] = B_{t,c}[k][j]   (inverse applies B^T: out j, in k)
+// both [d/b][b][kpad] floats, zero in the padding.
+struct StageDev {
+    int b;
+    int kpad;
+    int64_t s;
+    const float *fwd;
+    const float *inv;
+};
+
+struct PlanDev {
+    int64_t d;
+    int m;
+    const float *signs;  // [d] +-1 (always present; all ones when none given)
+    StageDev st[HARP_MAX_STAGES];
+};
+
+// Quantizer tables travel by value as a kernel argument.
+struct QuantDev {
+    int kind;       // HARP_LLOYD_MAX | HARP_ABSMAX
+    int bits;
+    int group;
+    float level[16];  // dequantised level per code (centroid or code - 2^(b-1))
+    float thr[16];    // Lloyd-Max midpoints (K - 1 used)
+};
+
+enum Prologue { PRO_F32 = 0, PRO_BF16 = 1, PRO_CODES = 2 };
+enum Epilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_QUANT = 2, EPI_QUANT_F32 = 3 };
+
+// Launch parameters of the whole-vector kernel: `nvec` vectors of length
+// plan.d taken from a row-major matrix, either its rows (side RIGHT) or its
+// columns (side LEFT).
+struct VecLaunch {
+    int side;
+    int dir;
+    int pro;
+    int epi;
+    int64_t nvec;
+    const void *in;
+    int64_t ld_in;
+    void *out;             // EPI_F32 / EPI_BF16 / EPI_QUANT_F32 (fp32 copy)
+    int64_t ld_out;
+    uint8_t *codes;        // EPI_QUANT*: packed codes, row stride = d*bits/8
+    uint16_t *scales;      // EPI_QUANT*: [nvec][d/group]
+    const uint8_t *in_codes;     // PRO_CODES
+    const uint16_t *in_scales;   // PRO_CODES
+};
+
+// Returns a cudaError_t value (0 = success).
+int launch_vec(const PlanDev &plan, const QuantDev *q, const VecLaunch &L, void *stream);
+int launch_quantize(const QuantDev &q, const void *in, int in_dtype, int64_t rows, int64_t cols,
+                    int64_t ld_in, uint8_t *codes, uint16_t *scales, void *stream);
+int launch_dequantize(const QuantDev &q, const uint8_t *codes, const uint16_t *scales,
+                      int64_t rows, int64_t cols, void *out, int out_dtype, int64_t ld_out,
+                      void *stream);
+
+// Vectors per CTA the whole-vector kernel would use for this shape (0 if the
+// vector does not fit in shared memory). Exposed for the tests and bench.
+int vec_tile(int64_t d, int epi, int group);
+
+}  // namespace harp

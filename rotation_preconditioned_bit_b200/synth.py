@@ -251,3 +251,15 @@ def small_matrix(seed: int, rows: int, cols: int, outlier_cols: int = 0,
     if outlier_cols:
         x[:, choose(seed, S_OUTLIER, cols, outlier_cols)] *= 20.0
     return x
+
+
+def random_code_stream(seed: int, rows: int, cols: int, bits: int, group: int,
+                       scale_lo: float = 0.01, scale_hi: float = 0.05):
+    """Random inputs for the inverse path: packed code bytes (any byte string
+    is a valid LSB-first code stream, so uniform bytes are uniform codes) and
+    fp16 scale bits uniform in [scale_lo, scale_hi)."""
+    nbytes = cols * bits // 8
+    raw = raw_u64(seed, 1, rows * nbytes).astype(np.uint8).reshape(rows, nbytes)
+    u = uniform(seed, 2, rows * (cols // group)).reshape(rows, cols // group)
+    sc = (scale_lo + (scale_hi - scale_lo) * u).astype(np.float16).view(np.uint16)
+    return raw, sc

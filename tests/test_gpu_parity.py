@@ -1,0 +1,317 @@
+"""GPU-vs-oracle parity of the CUDA path, called through the C ABI.
+
+Every input comes from the seeded generator (synth); the oracle builds its own
+float64 blocks and codebook from the same raw draws. Full-size workloads are
+compared element by element where the oracle finishes in seconds (the
+64x256, 4096x4096 and [T, 4096] workloads) and on sampled rows otherwise
+(4096x11008, 8192x28672), in the launch configuration the benchmark times.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from parity import TOL_BF16, TOL_F32, compare_quant, np_unpack, rel_l2
+from rotation_preconditioned_bit_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import rotation_preconditioned_bit_b200 as harp
+
+
+_WL = {}
+
+
+def wl(name, **kw):
+    key = (name, tuple(sorted(kw.items())))
+    if key not in _WL:
+        _WL[key] = synth.workload(name, **kw)
+    return _WL[key]
+
+
+def to_dev(w):
+    if w.dtype == "bf16":
+        return torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(w.x)).cuda()
+
+
+def scales_np(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def sample_rows(rows, n, seed):
+    pick = synth.choose(seed, 77, rows, n - 3)
+    return np.unique(np.concatenate([[0, rows // 2, rows - 1], pick])).astype(np.int64)
+
+
+# ------------------------------------------------------------ 64 x 256 fp32, (16,16) Sylvester
+
+def test_c1_rotate_matches_oracle():
+    w = wl("c1")
+    P = oracle.processor(w.right)
+    ref = P.rotate_rows(synth.x_as_f64(w))
+    plan = harp.Plan.from_side(w.right)
+    x = to_dev(w)
+    out = torch.empty_like(x)
+    harp.harp_rotate(plan, harp.HARP_RIGHT, harp.HARP_FWD, x, out)
+    assert rel_l2(out.cpu().numpy(), ref) <= TOL_F32
+    back = torch.empty_like(x)
+    harp.harp_rotate(plan, harp.HARP_RIGHT, harp.HARP_INV, out, back)
+    assert rel_l2(back.cpu().numpy(), synth.x_as_f64(w)) <= TOL_F32
+
+
+def test_c1_rotate_quantize_matches_oracle():
+    w = wl("c1")
+    q = w.quants[0]
+    P = oracle.processor(w.right)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(synth.x_as_f64(w), None, P, q.kind, q.bits, q.group)
+    plan = harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    codes, scales, rot = harp.rotate_quantize(None, plan, cb, to_dev(w), want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    rep = compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, q.bits, q.group)
+    assert rep["near_boundary"] < 0.001 * rep["elements"]
+
+
+# ------------------------------------------------------------ 4096 x 4096 bf16, two-sided
+
+@pytest.fixture(scope="module")
+def c2_ref():
+    w = wl("c2")
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    return w, Pr.rotate_rows(Pl.rotate_cols(synth.x_as_f64(w)))
+
+
+@pytest.mark.parametrize("qi", [0, 1])
+def test_c2_two_sided_full_matrix(c2_ref, qi):
+    w, ref = c2_ref
+    q = w.quants[qi]
+    oc, osc, m, sm = oracle.quantize(q.kind, q.bits, q.group, ref)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    x = to_dev(w)
+    codes, scales, rot = harp.rotate_quantize(left, right, cb, x, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    rep = compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, q.bits, q.group)
+    print(f"\nc2 {q.kind} {q.bits}-bit:", rep)
+    # the benchmark's call (no fp32 copy) gives the same bytes
+    codes2, scales2, _ = harp.rotate_quantize(left, right, cb, x)
+    assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
+
+
+def test_c2_unfused_equals_fused(c2_ref):
+    w, _ = c2_ref
+    q = w.quants[1]
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    x = to_dev(w)
+    codes, scales, _ = harp.rotate_quantize(left, right, cb, x)
+    t = torch.empty(x.shape, dtype=torch.float32, device="cuda")
+    harp.harp_rotate(left, harp.HARP_LEFT, harp.HARP_FWD, x, t)
+    t2 = torch.empty_like(t)
+    harp.harp_rotate(right, harp.HARP_RIGHT, harp.HARP_FWD, t, t2)
+    c2, s2 = harp.empty_codes(*x.shape, cb)
+    harp.harp_quantize(cb, t2, c2, s2)
+    assert torch.equal(c2, codes) and torch.equal(s2, scales)
+
+
+# ------------------------------------------------------------ [T, 4096] activations, per-token absmax
+
+@pytest.mark.parametrize("T", [1, 16, 256, 8192])
+def test_c3_activation_rows(T):
+    w = wl("c3", tokens=T)
+    q = w.quants[0]
+    P = oracle.processor(w.right)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(synth.x_as_f64(w), None, P, q.kind, q.bits, q.group)
+    plan = harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    codes, scales, rot = harp.rotate_quantize(None, plan, cb, to_dev(w), want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, q.bits, q.group)
+    # bf16 rotated activations
+    xb = torch.empty((T, 4096), dtype=torch.bfloat16, device="cuda")
+    harp.harp_rotate(plan, harp.HARP_RIGHT, harp.HARP_FWD, to_dev(w), xb)
+    assert rel_l2(xb.float().cpu().numpy(), ref) <= TOL_BF16
+
+
+# ------------------------------------------------------------ sampled rows of the large workloads
+
+def _sampled_forward(w, q, which):
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    X = synth.x_as_f64(w)
+    ref = oracle.two_sided_rows(X, Pl, Pr, which)
+    oc, osc, m, sm = oracle.quantize(q.kind, q.bits, q.group, ref)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    x = to_dev(w)
+    codes, scales, rot = harp.rotate_quantize(left, right, cb, x, want_rotated=True)
+    idx = torch.from_numpy(which).cuda()
+    assert rel_l2(rot[idx].cpu().numpy(), ref) <= TOL_F32
+    rep = compare_quant(codes[idx].cpu().numpy(), scales_np(scales[idx]), oc, osc, m, sm, q.bits, q.group)
+    codes2, scales2, _ = harp.rotate_quantize(left, right, cb, x)
+    assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
+    return left, right, cb, codes, scales, rep
+
+
+def _sampled_inverse(w, q, which, seed):
+    """Random packed bytes and scales (any byte string is a valid code
+    stream) through dequantize + inverse rotation, against the oracle."""
+    rows, cols = w.rows, w.cols
+    raw, sc = synth.random_code_stream(seed, rows, cols, q.bits, q.group)
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    Wp = oracle.dequantize(q.kind, q.bits, q.group, oracle.unpack(q.bits, raw, cols), sc)
+    ref = oracle.inverse_rows(Wp, Pl, Pr, which)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    codes = torch.from_numpy(raw).cuda()
+    scales = torch.from_numpy(sc.view(np.int16)).cuda()
+    out = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.float32)
+    idx = torch.from_numpy(which).cuda()
+    assert rel_l2(out[idx].cpu().numpy(), ref) <= TOL_F32
+    outb = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.bfloat16)
+    assert rel_l2(outb[idx].float().cpu().numpy(), ref) <= TOL_BF16
+    # standalone dequantise of the same bytes
+    deq = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    harp.harp_dequantize(cb, codes, scales, deq)
+    np.testing.assert_allclose(deq[idx].cpu().numpy(), Wp[which], rtol=0, atol=1e-6 * np.abs(Wp).max())
+
+
+def test_c4_forward_sampled_and_round_trip():
+    w = wl("c4")
+    q = w.quants[0]
+    which = sample_rows(w.rows, 12, 41)
+    left, right, cb, codes, scales, rep = _sampled_forward(w, q, which)
+    print("\nc4 3-bit:", rep)
+    # round trip: an exact change of basis keeps the error norm
+    What = harp.dequantize_unrotate(left, right, cb, codes, scales, w.rows, w.cols, torch.float32)
+    Wp_hat = torch.empty((w.rows, w.cols), dtype=torch.float32, device="cuda")
+    harp.harp_dequantize(cb, codes, scales, Wp_hat)
+    x = to_dev(w).float()
+    _, _, rot = harp.rotate_quantize(left, right, cb, to_dev(w), want_rotated=True)
+    e_orig = torch.linalg.norm((x - What).double()).item()
+    e_rot = torch.linalg.norm((rot - Wp_hat).double()).item()
+    assert abs(e_orig - e_rot) <= 1e-5 * e_rot
+
+
+def test_c4_inverse_sampled():
+    w = wl("c4")
+    _sampled_inverse(w, w.quants[0], sample_rows(w.rows, 10, 43), 4040)
+
+
+@pytest.mark.parametrize("qi", [0, 1])
+def test_c5_forward_sampled(qi):
+    w = wl("c5")
+    q = w.quants[qi]
+    which = sample_rows(w.rows, 8, 51 + qi)
+    rep = _sampled_forward(w, q, which)[-1]
+    print(f"\nc5 {q.kind} {q.bits}-bit:", rep)
+
+
+@pytest.mark.parametrize("qi", [0, 1])
+def test_c5_inverse_sampled(qi):
+    w = wl("c5")
+    _sampled_inverse(w, w.quants[qi], sample_rows(w.rows, 6, 61 + qi), 5050 + qi)
+
+
+# ------------------------------------------------------------ small shapes, every radix path
+
+RADICES = [(2, 4), (4, 4), (8, 2, 4), (3, 5), (7,), (16, 16), (5, 3, 2), (64, 4), (43, 2),
+           (2, 2, 2, 2, 2, 2), (1, 8), (6, 6), (32, 16, 16)]
+
+
+@pytest.mark.parametrize("radix", RADICES)
+@pytest.mark.parametrize("side", ["right", "left"])
+def test_small_rotate_both_directions(radix, side):
+    d = int(np.prod(radix))
+    s = synth.side_draws(700 + d, radix, "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    P = oracle.processor(s)
+    plan = harp.Plan.from_side(s)
+    nvec = 37                                  # ragged against every tile size
+    if side == "right":
+        X = synth.small_matrix(d, nvec, d)
+        sd, rot = harp.HARP_RIGHT, P.rotate_rows
+        buf_shape, view = (nvec, ((d + 3) // 4) * 4), (slice(None), slice(0, d))
+    else:
+        X = synth.small_matrix(d, d, nvec)
+        sd, rot = harp.HARP_LEFT, P.rotate_cols
+        buf_shape, view = (d, 40), (slice(None), slice(0, nvec))
+    Xf = X.astype(np.float32).astype(np.float64)
+    xb = torch.zeros(buf_shape, dtype=torch.float32, device="cuda")
+    xv = xb[view]
+    xv.copy_(torch.from_numpy(X.astype(np.float32)))
+    ob = torch.full(buf_shape, 7.0, dtype=torch.float32, device="cuda")
+    ov = ob[view]
+    harp.harp_rotate(plan, sd, harp.HARP_FWD, xv, ov)
+    assert rel_l2(ov.cpu().numpy(), rot(Xf)) <= TOL_F32
+    # padding outside the view is untouched
+    mask = torch.ones(buf_shape, dtype=torch.bool, device="cuda")
+    mask[view] = False
+    assert torch.all(ob[mask] == 7.0)
+    harp.harp_rotate(plan, sd, harp.HARP_INV, xv, ov)
+    assert rel_l2(ov.cpu().numpy(), rot(Xf, inverse=True)) <= TOL_F32
+    # bf16 in, bf16 out (padded leading dimension)
+    x16b = torch.zeros(buf_shape, dtype=torch.bfloat16, device="cuda")
+    x16 = x16b[view]
+    x16.copy_(xv)
+    X16 = x16.float().cpu().numpy().astype(np.float64)
+    o16b = torch.zeros(buf_shape, dtype=torch.bfloat16, device="cuda")
+    o16 = o16b[view]
+    harp.harp_rotate(plan, sd, harp.HARP_FWD, x16, o16)
+    assert rel_l2(o16.float().cpu().numpy(), rot(X16)) <= TOL_BF16
+    # bf16 in, fp32 out is exact-input fp32 arithmetic
+    harp.harp_rotate(plan, sd, harp.HARP_FWD, x16, ov)
+    assert rel_l2(ov.cpu().numpy(), rot(X16)) <= TOL_F32
+
+
+@pytest.mark.parametrize("kind,bits,group", [("lloyd_max", 2, 32), ("lloyd_max", 3, 64),
+                                             ("lloyd_max", 4, 128), ("absmax", 2, 64),
+                                             ("absmax", 3, 512), ("absmax", 4, 32)])
+def test_standalone_quantize_and_dequantize(kind, bits, group):
+    rows, cols = 33, 512
+    X = synth.small_matrix(bits * 10 + group, rows, cols, outlier_cols=3, scale=0.02)
+    X32 = X.astype(np.float32)
+    oc, osc, m, sm = oracle.quantize(kind, bits, group, X32.astype(np.float64))
+    cb = harp.Codebook(kind, bits, group)
+    x = torch.from_numpy(X32).cuda()
+    codes, scales = harp.empty_codes(rows, cols, cb)
+    harp.harp_quantize(cb, x, codes, scales)
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+    deq = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    harp.harp_dequantize(cb, codes, scales, deq)
+    gc = np_unpack(codes.cpu().numpy(), bits, cols)
+    ref = oracle.dequantize(kind, bits, group, oc, osc)
+    same = (gc == oc) & (scales_np(scales) == osc).repeat(group, axis=1)
+    np.testing.assert_allclose(deq.cpu().numpy()[same], ref[same], rtol=1e-7, atol=0)
+
+
+def test_edge_cases_zero_rows_huge_values_and_empty():
+    cb = harp.Codebook("lloyd_max", 4, 128)
+    X = np.zeros((3, 256), np.float32)
+    X[1, :128] = 1e6            # RMS above the fp16 range: scale saturates at 65504
+    X[2] = synth.small_matrix(3, 1, 256)[0]
+    oc, osc, m, sm = oracle.quantize("lloyd_max", 4, 128, X.astype(np.float64))
+    codes, scales = harp.empty_codes(3, 256, cb)
+    harp.harp_quantize(cb, torch.from_numpy(X).cuda(), codes, scales)
+    s = scales_np(scales)
+    assert s[0, 0] == 0 and s[0, 1] == 0 and s[1, 0] == 0x7BFF
+    compare_quant(codes.cpu().numpy(), s, oc, osc, m, sm, 4, 128)
+    gc = np_unpack(codes.cpu().numpy(), 4, 256)
+    assert np.all(gc[0] == 8)
+    # empty matrices launch nothing and succeed
+    s16 = synth.side_draws(1, (16, 16), "hadamard", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    plan = harp.Plan.from_side(s16)
+    e = torch.empty((0, 256), dtype=torch.float32, device="cuda")
+    c0, sc0 = harp.empty_codes(0, 256, cb)
+    harp.harp_rotate_quantize(None, plan, cb, e, c0, sc0)
+    harp.harp_rotate(plan, harp.HARP_RIGHT, harp.HARP_FWD, e, torch.empty_like(e))
+    torch.cuda.synchronize()
+
+
+def test_plan_info_and_workspace():
+    s = synth.side_draws(5, (43, 16, 16), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    plan = harp.Plan.from_side(s)
+    assert plan.info() == (11008, 3, (43, 16, 16))
+    assert harp.workspace_size(plan, plan, 11008, 11008) == 11008 * 11008 * 4
+    assert harp.workspace_size(None, plan, 7, 11008) == 0
