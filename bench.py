@@ -26,6 +26,8 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import shutil
+import signal
 import statistics
 import subprocess
 import sys
@@ -90,10 +92,13 @@ class ClockSampler:
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            cmd = ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                   "--format=csv,noheader,nounits", "-lms", "20"]
+            if shutil.which("stdbuf"):
+                cmd = ["stdbuf", "-oL"] + cmd      # line-buffered: samples arrive as taken
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            time.sleep(0.3)                         # first sample before the timed region
         except Exception:
             self.proc = None
             return
@@ -107,7 +112,8 @@ class ClockSampler:
     def stop(self):
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
+        time.sleep(0.05)
+        self.proc.send_signal(signal.SIGINT)
         try:
             self.proc.wait(timeout=5)
         except Exception:

@@ -465,7 +465,7 @@ static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, i
     if (st) return st;
     if (right->d != cols) return HARP_ERR_SHAPE;
     if (left && left->d != rows) return HARP_ERR_SHAPE;
-    if (harp::vec_tile(cols, harp::EPI_QUANT, cb->q.group) == 0) return HARP_ERR_UNSUPPORTED;
+    if (harp::vec_tile(right->dev, harp::EPI_QUANT, cb->q.group) == 0) return HARP_ERR_UNSUPPORTED;
     if (left) {
         const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(cols) * 4;
         if (need && (!workspace || ws_bytes < need)) return HARP_ERR_WORKSPACE;

@@ -69,8 +69,8 @@ int launch_dequantize(const QuantDev &q, const uint8_t *codes, const uint16_t *s
                       int64_t rows, int64_t cols, void *out, int out_dtype, int64_t ld_out,
                       void *stream);
 
-// Vectors per CTA the whole-vector kernel would use for this shape (0 if the
-// vector does not fit in shared memory). Exposed for the tests and bench.
-int vec_tile(int64_t d, int epi, int group);
+// Vectors per CTA the whole-vector kernel uses for this plan and epilogue
+// (0 if a vector does not fit in shared memory).
+int vec_tile(const PlanDev &plan, int epi, int group);
 
 }  // namespace harp

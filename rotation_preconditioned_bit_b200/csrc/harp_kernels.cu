@@ -30,7 +30,7 @@
 namespace harp {
 namespace {
 
-constexpr int NT = 512;              // threads per CTA
+constexpr int NT = 256;              // threads per CTA (up to 255 registers each)
 constexpr int SMEM_MAX = 232448;     // opt-in dynamic shared memory per CTA (227 KB)
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -139,33 +139,237 @@ __device__ __forceinline__ unsigned short group_scale_bits(float stat, const Qua
     return __half_as_ushort(__float2half_rn(s));
 }
 
-// Code of one value given its group's stored scale (as float) and the fp32
-// midpoint table (Lloyd-Max: number of midpoints below x/s; absmax: rounded
-// and clamped x/s, offset by 2^(b-1)). A zero scale gives the middle code.
-__device__ __forceinline__ int quant_code(float x, float s, const QuantDev &Q, const float *thr) {
-    const int half = 1 << (Q.bits - 1);
-    if (!(s > 0.0f)) return half;
-    const float z = x * __frcp_rn(s);
-    if (Q.kind == HARP_LLOYD_MAX) {
-        int code = 0;
-        for (int step = half; step >= 1; step >>= 1)
-            if (z > thr[code + step - 1]) code += step;
-        return code;
+// ------------------------------------------------------------ tile geometry
+
+// Shared-memory tile of R vectors: coordinate i's R floats start at
+//   row(i) = i * Rp + padq * (i / bl)
+// with bl the last radix of the schedule. The 4-float pad after every last-
+// radix group puts neighbouring groups of the last stage (which are bl
+// coordinates apart) on different banks; every stage's group then has an
+// affine address a0 + j * Sj in its input index j.
+struct Geo {
+    int d, R, Rp, padq, bl, bl_shift;
+    __device__ __forceinline__ int div_bl(int i) const { return bl_shift >= 0 ? (i >> bl_shift) : (i / bl); }
+    __device__ __forceinline__ int row(int i) const { return i * Rp + padq * div_bl(i); }
+};
+
+// ------------------------------------------------------------ stage core
+
+template <int VW>
+__device__ __forceinline__ void ldsv(const float *p, float (&v)[VW]) {
+    if constexpr (VW == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else if constexpr (VW == 2) {
+        const float2 t = *reinterpret_cast<const float2 *>(p);
+        v[0] = t.x; v[1] = t.y;
+    } else {
+        v[0] = *p;
     }
-    const float qmax = static_cast<float>(half - 1);
-    const float q = fminf(fmaxf(rintf(z), -qmax), qmax);
-    return static_cast<int>(q) + half;
 }
 
-// Pack the warp's 32 consecutive codes (lane = position) into `bits` 32-bit
-// words of the LSB-first bitstream; returns word `lane` (valid for lane < bits).
-__device__ __forceinline__ unsigned pack_warp(int code, int bits, int lane) {
-    const int bit0 = bits * lane;
+template <int VW>
+__device__ __forceinline__ void stsv(float *p, const float *v) {
+    if constexpr (VW == 4) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (VW == 2) {
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    } else {
+        *p = v[0];
+    }
+}
+
+// Coefficients j0 .. j0+CJ-1 of rows k0 .. k0+KL-1 of group c: for the
+// forward direction rows of B (output k, inputs j), for the inverse columns
+// of B. Rows past b, inputs past b and groups past the end read as zero.
+constexpr int CJ = 8;   // inputs per coefficient chunk
+
+template <int KL>
+__device__ __forceinline__ void load_chunk(const float *__restrict__ rows, int c, int ngroups, int b,
+                                           int kpad, int k0, int j0, bool active, float (&dst)[KL][CJ]) {
+#pragma unroll
+    for (int k = 0; k < KL; ++k) {
+        const bool ok = active && (c < ngroups) && (k0 + k < b);
+        const float4 *p = reinterpret_cast<const float4 *>(
+            rows + (static_cast<size_t>(ok ? c : 0) * b + (ok ? k0 + k : 0)) * kpad + j0);
+#pragma unroll
+        for (int q = 0; q < CJ / 4; ++q) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ok && j0 + q * 4 < b) v = __ldg(p + q);
+            dst[k][4 * q + 0] = v.x; dst[k][4 * q + 1] = v.y;
+            dst[k][4 * q + 2] = v.z; dst[k][4 * q + 3] = v.w;
+        }
+    }
+}
+
+// acc[k][v] += sum_{j < jn} w[k][j] * X[a + j*Sj + v] for one chunk of <= CJ
+// inputs. FULL chunks carry no per-input guard: a guard inside the unrolled
+// loop keeps the compiler from scheduling the shared loads ahead of the FMAs
+// and halves the FMA rate.
+template <int VW, int NV, int KL, bool FULL>
+__device__ __forceinline__ void chunk_fma(const float *X, int a, int Sj, int jn, const float (&w)[KL][CJ],
+                                          float (&acc)[KL][VW * NV]) {
+#pragma unroll
+    for (int j = 0; j < CJ; ++j) {
+        if (FULL || j < jn) {
+            const float *xp = X + a + j * Sj;
+            float x[NV][VW];
+#pragma unroll
+            for (int n = 0; n < NV; ++n) ldsv<VW>(xp + n * VW, x[n]);
+#pragma unroll
+            for (int k = 0; k < KL; ++k) {
+                const float wk = w[k][j];
+#pragma unroll
+                for (int n = 0; n < NV; ++n)
+#pragma unroll
+                    for (int e = 0; e < VW; ++e) acc[k][n * VW + e] = fmaf(wk, x[n][e], acc[k][n * VW + e]);
+            }
+        }
+    }
+}
+
+// Per-stage constants of the coefficient stream of one thread.
+struct StageIt {
+    const float *rows;
+    int b, kpad, s, s_shift, Sj, k0, qi, Gr, ngroups, nc;
+    bool active;
+};
+
+// One element e of the thread's coefficient stream: chunk (e % nc) of round
+// (e / nc). Prefetches element e+1 into `nxt`, accumulates this chunk from
+// `cur`; after a round's last chunk: barrier, then the outputs are written
+// in place over the group's inputs.
+template <int VW, int NV, int KL>
+__device__ __forceinline__ void stream_step(float *X, const Geo &g, const StageIt &it, int e, int total,
+                                            float (&cur)[KL][CJ], float (&nxt)[KL][CJ],
+                                            float (&acc)[KL][VW * NV], int &a0) {
+    const int r = e / it.nc, ch = e - r * it.nc;
+    if (e + 1 < total) {
+        const int r1 = (ch + 1 == it.nc) ? r + 1 : r;
+        const int ch1 = (ch + 1 == it.nc) ? 0 : ch + 1;
+        load_chunk<KL>(it.rows, r1 * it.Gr + it.qi, it.ngroups, it.b, it.kpad, it.k0, ch1 * CJ, it.active, nxt);
+    }
+    const int c = r * it.Gr + it.qi;
+    const bool ok = it.active && (c < it.ngroups);
+    if (ch == 0) {
+#pragma unroll
+        for (int k = 0; k < KL; ++k)
+#pragma unroll
+            for (int v = 0; v < VW * NV; ++v) acc[k][v] = 0.0f;
+        if (ok) {
+            const int h = (it.s_shift >= 0) ? (c >> it.s_shift) : (c / it.s);
+            const int l = c - h * it.s;
+            a0 = g.row(h * it.b * it.s + l);
+        }
+    }
+    if (ok) {
+        const int jn = it.b - ch * CJ;
+        if (jn >= CJ) chunk_fma<VW, NV, KL, true>(X, a0 + ch * CJ * it.Sj, it.Sj, CJ, cur, acc);
+        else chunk_fma<VW, NV, KL, false>(X, a0 + ch * CJ * it.Sj, it.Sj, jn, cur, acc);
+    }
+    if (ch + 1 == it.nc) {
+        __syncthreads();
+        if (ok) {
+#pragma unroll
+            for (int k = 0; k < KL; ++k) {
+                if (it.k0 + k < it.b) {
+                    float *yp = X + a0 + (it.k0 + k) * it.Sj;
+#pragma unroll
+                    for (int n = 0; n < NV; ++n) stsv<VW>(yp + n * VW, &acc[k][n * VW]);
+                }
+            }
+        }
+    }
+}
+
+// One stride stage over the whole tile. Each thread owns KL consecutive
+// outputs of one group per round (all R vectors of the tile); groups are
+// handed out Gr = NT / ceil(b / KL) per round. The thread's coefficients
+// arrive as a stream of CJ-input chunks, always one chunk ahead.
+template <int VW, int NV, int KL>
+__device__ __forceinline__ void stage_core(float *X, const Geo &g, const StageDev &S, bool last,
+                                           int dir, int tid) {
+    StageIt it;
+    it.b = S.b;
+    it.kpad = S.kpad;
+    it.s = static_cast<int>(S.s);
+    it.s_shift = (it.s & (it.s - 1)) == 0 ? __ffs(it.s) - 1 : -1;
+    const int npairs = (it.b + KL - 1) / KL;
+    it.Gr = NT / npairs;
+    it.ngroups = g.d / it.b;
+    it.qi = tid / npairs;
+    it.k0 = (tid - it.qi * npairs) * KL;
+    it.active = it.qi < it.Gr;
+    it.Sj = last ? g.Rp : it.s * g.Rp + g.padq * g.div_bl(it.s);
+    it.rows = (dir == HARP_FWD) ? S.inv : S.fwd;
+    it.nc = (it.b + CJ - 1) / CJ;
+    const int nrounds = (it.ngroups + it.Gr - 1) / it.Gr;
+    const int total = nrounds * it.nc;
+    float bufA[KL][CJ], bufB[KL][CJ], acc[KL][VW * NV];
+    int a0 = 0;
+    load_chunk<KL>(it.rows, it.qi, it.ngroups, it.b, it.kpad, it.k0, 0, it.active, bufA);
+    for (int e = 0; e < total; e += 2) {
+        stream_step<VW, NV, KL>(X, g, it, e, total, bufA, bufB, acc, a0);
+        if (e + 1 < total) stream_step<VW, NV, KL>(X, g, it, e + 1, total, bufB, bufA, acc, a0);
+    }
+    __syncthreads();
+}
+
+template <int VW, int NV>
+__device__ __forceinline__ void run_stage(float *X, const Geo &g, const StageDev &S, bool last, int dir, int tid) {
+    // outputs per thread: enough FMAs per shared load, registers permitting
+    constexpr int R = VW * NV;
+    constexpr int KL = (R <= 12) ? 4 : 2;
+    stage_core<VW, NV, KL>(X, g, S, last, dir, tid);
+}
+
+// ------------------------------------------------------------ quantizer epilogue
+
+// t[OFF + STRIDE * idx] for idx in [0, N) (N a power of two) by a tree of
+// selects on the bits of idx: the array stays in registers.
+template <int OFF, int N, int STRIDE, int K>
+__device__ __forceinline__ float pick(const float (&t)[K], int idx) {
+    if constexpr (N == 1) {
+        return t[OFF];
+    } else {
+        return (idx & (N / 2)) ? pick<OFF + STRIDE * (N / 2), N / 2, STRIDE, K>(t, idx)
+                               : pick<OFF, N / 2, STRIDE, K>(t, idx);
+    }
+}
+
+// Lloyd-Max code = number of midpoints below z: binary search over the
+// sorted fp32 midpoints held in registers (ties go to the lower code).
+template <int BITS, int STEP = (1 << (BITS - 1))>
+__device__ __forceinline__ int lm_search(float z, const float (&t)[(1 << BITS) - 1], int code) {
+    if constexpr (STEP == 0) {
+        return code;
+    } else {
+        constexpr int K = 1 << BITS;
+        const float th = pick<STEP - 1, K / (2 * STEP), 2 * STEP, K - 1>(t, code / (2 * STEP));
+        return lm_search<BITS, STEP / 2>(z, t, code + ((z > th) ? STEP : 0));
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ int code_of(float x, float s, float inv_s, bool lloyd,
+                                       const float (&t)[(1 << BITS) - 1]) {
+    constexpr int HALF = 1 << (BITS - 1);
+    if (!(s > 0.0f)) return HALF;
+    const float z = x * inv_s;
+    if (lloyd) return lm_search<BITS>(z, t, 0);
+    const float qmax = static_cast<float>(HALF - 1);
+    return static_cast<int>(fminf(fmaxf(rintf(z), -qmax), qmax)) + HALF;
+}
+
+template <int BITS>
+__device__ __forceinline__ unsigned pack_words(int code, int lane) {
+    const int bit0 = BITS * lane;
     const int wlo = bit0 >> 5, sh = bit0 & 31;
     const unsigned lo = static_cast<unsigned>(code) << sh;
-    const unsigned hi = (sh + bits > 32) ? (static_cast<unsigned>(code) >> (32 - sh)) : 0u;
+    const unsigned hi = (sh + BITS > 32) ? (static_cast<unsigned>(code) >> (32 - sh)) : 0u;
     unsigned mine = 0;
-    for (int w = 0; w < bits; ++w) {
+#pragma unroll
+    for (int w = 0; w < BITS; ++w) {
         const unsigned part = (w == wlo ? lo : 0u) | (w == wlo + 1 ? hi : 0u);
         const unsigned word = __reduce_or_sync(FULL, part);
         if (w == lane) mine = word;
@@ -173,195 +377,264 @@ __device__ __forceinline__ unsigned pack_warp(int code, int bits, int lane) {
     return mine;
 }
 
-// ------------------------------------------------------------ stage core
+// Group statistic of `g` consecutive values for one vector: each lane
+// accumulates its values (coordinates lane, lane+32, ...) in order, then a
+// fixed xor tree combines the lanes. The standalone quantizer uses the same
+// order, so both give identical scales.
+__device__ __forceinline__ float combine(float a, float x, bool is_max) {
+    return is_max ? fmaxf(a, fabsf(x)) : fmaf(x, x, a);
+}
 
-// One stride stage on the shared tile X[coord * Rp + vector] (R vectors).
-// A unit is (group, 4 consecutive outputs, BT consecutive vectors); units of
-// whole groups are handed out round by round.
-template <int BT>
-__device__ __forceinline__ void run_stage(float *X, int Rp, int R, int d, const StageDev &S,
-                                          int dir, int tid) {
-    constexpr int UPT = (BT == 4) ? 4 : 8;   // units per thread per round
-    const int b = S.b, kpad = S.kpad, nk = kpad >> 2;
-    const int s = static_cast<int>(S.s);
-    const float *__restrict__ A = (dir == HARP_FWD) ? S.fwd : S.inv;
-    const int nbq = R / BT;
-    const int Ug = nk * nbq;          // units per group
-    const int ngroups = d / b;
-    int Gr = (UPT * NT) / Ug;         // whole groups per round
-    if (Gr < 1) Gr = 1;
-    const int sRp = s * Rp;
-
-    for (int g0 = 0; g0 < ngroups; g0 += Gr) {
-        const int gcount = min(Gr, ngroups - g0);
-        const int nunits = gcount * Ug;
-        float acc[UPT][4][BT];
-        int aoff[UPT], xoff[UPT], sk[UPT];
+// Scales and codes of the tile's rows (forward, rows side).
+template <int VW, int BITS, bool F32OUT>
+__device__ __forceinline__ void quantize_tile(const float *X, const Geo &g, const QuantDev &Q,
+                                              float *sc, float *isc, const VecLaunch &L, int64_t v0,
+                                              int warp, int lane) {
+    constexpr int NWARP = NT / 32;
+    const int d = g.d, gsz = Q.group, ng = d / gsz, nchunk = d >> 5, cpg = gsz >> 5;
+    const int nrv = g.R / VW;
+    const bool is_max = (Q.kind == HARP_ABSMAX);
+    const bool lloyd = !is_max;
+    // pass 1: statistics and scales, one (row group of VW rows, scale group) per warp
+    for (int item = warp; item < nrv * ng; item += NWARP) {
+        const int gi = item / nrv, rq = item - gi * nrv;
+        float st[VW];
 #pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int unit = tid + u * NT;
-            const int uu = (unit < nunits) ? unit : 0;
-            const int q = uu / Ug;
-            const int rem = uu - q * Ug;
-            const int kq = rem / nbq;
-            const int bq = rem - kq * nbq;
-            const int c = g0 + q;
-            const int h = c / s;
-            const int l = c - h * s;
-            aoff[u] = c * b * kpad + kq * 4;
-            xoff[u] = (h * b * s + l) * Rp + bq * BT;
-            sk[u] = q % b;           // skew the j order per group: spreads smem banks
+        for (int v = 0; v < VW; ++v) st[v] = 0.0f;
+#pragma unroll 4
+        for (int c = 0; c < cpg; ++c) {
+            float x[VW];
+            ldsv<VW>(X + g.row(gi * gsz + c * 32 + lane) + rq * VW, x);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int v = 0; v < BT; ++v) acc[u][k][v] = 0.0f;
+            for (int v = 0; v < VW; ++v) st[v] = combine(st[v], x[v], is_max);
         }
-#pragma unroll 1
-        for (int jj = 0; jj < b; ++jj) {
 #pragma unroll
-            for (int u = 0; u < UPT; ++u) {
-                int j = jj + sk[u];
-                j -= (j >= b) ? b : 0;
-                const float4 a = __ldg(reinterpret_cast<const float4 *>(A + aoff[u] + j * kpad));
-                float x[BT];
-                lds<BT>(X + xoff[u] + j * sRp, x);
-#pragma unroll
-                for (int v = 0; v < BT; ++v) {
-                    acc[u][0][v] = fmaf(a.x, x[v], acc[u][0][v]);
-                    acc[u][1][v] = fmaf(a.y, x[v], acc[u][1][v]);
-                    acc[u][2][v] = fmaf(a.z, x[v], acc[u][2][v]);
-                    acc[u][3][v] = fmaf(a.w, x[v], acc[u][3][v]);
-                }
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int unit = tid + u * NT;
-            if (unit < nunits) {
-                const int kq4 = ((unit % Ug) / nbq) * 4;
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (kq4 + k < b) sts<BT>(X + xoff[u] + (kq4 + k) * sRp, acc[u][k]);
+        for (int v = 0; v < VW; ++v) {
+            const float tot = warp_reduce(st[v], is_max);
+            if (lane == v) {
+                const int r = rq * VW + v;
+                const unsigned short hb = group_scale_bits(tot, Q);
+                const float sv = __half2float(__ushort_as_half(hb));
+                sc[r * ng + gi] = sv;
+                isc[r * ng + gi] = (sv > 0.0f) ? __frcp_rn(sv) : 0.0f;
+                const int64_t row = v0 + r;
+                if (row < L.nvec) L.scales[row * ng + gi] = hb;
             }
         }
     }
     __syncthreads();
+    // pass 2: codes and packing, one (row group, 32-coordinate chunk) per warp
+    float t[(1 << BITS) - 1];
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) t[k] = Q.thr[k];
+    const int64_t rowbytes = static_cast<int64_t>(d) * BITS / 8;
+    for (int item = warp; item < nrv * nchunk; item += NWARP) {
+        const int ch = item / nrv, rq = item - ch * nrv;
+        const int i = ch * 32 + lane;
+        const int gi = ch / cpg;
+        float x[VW];
+        ldsv<VW>(X + g.row(i) + rq * VW, x);
+#pragma unroll
+        for (int v = 0; v < VW; ++v) {
+            const int r = rq * VW + v;
+            const int64_t row = v0 + r;
+            const int code = code_of<BITS>(x[v], sc[r * ng + gi], isc[r * ng + gi], lloyd, t);
+            const unsigned word = pack_words<BITS>(code, lane);
+            if (row < L.nvec) {
+                if (lane < BITS)
+                    reinterpret_cast<unsigned *>(L.codes + row * rowbytes)[ch * BITS + lane] = word;
+                if constexpr (F32OUT) static_cast<float *>(L.out)[row * L.ld_out + i] = x[v];
+            }
+        }
+    }
+}
+
+// Dequantise R rows of packed codes into the tile (inverse path). One item
+// is 32 consecutive codes of one row: `BITS` aligned 32-bit words and one
+// scale (groups are multiples of 32 codes); items of neighbouring rows go to
+// neighbouring threads so the shared-memory writes are contiguous.
+template <int BITS>
+__device__ __forceinline__ void load_codes(float *X, const Geo &g, const QuantDev &Q, const VecLaunch &L,
+                                           const float *lev, int64_t v0, int tid) {
+    constexpr int IB = 4;
+    constexpr unsigned MASK = (1u << BITS) - 1u;
+    const int d = g.d, R = g.R, gsz = Q.group, ng = d / gsz;
+    const int nch = d >> 5;
+    const int n = R * nch;
+    const int64_t rowwords = static_cast<int64_t>(d) * BITS / 32;
+    for (int base = tid; base < n; base += NT * IB) {
+        unsigned w[IB][BITS];
+        float sc[IB];
+#pragma unroll
+        for (int u = 0; u < IB; ++u) {
+            const int idx = base + u * NT;
+            const int ch = idx / R, r = idx - ch * R;
+            const int64_t row = v0 + r;
+            const bool ok = idx < n && row < L.nvec;
+            const unsigned *src = reinterpret_cast<const unsigned *>(L.in_codes) + (ok ? row * rowwords + ch * BITS : 0);
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) w[u][q] = ok ? __ldg(src + q) : 0u;
+            sc[u] = ok ? __half2float(__ushort_as_half(__ldg(L.in_scales + row * ng + (ch * 32) / gsz))) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < IB; ++u) {
+            const int idx = base + u * NT;
+            if (idx < n) {
+                const int ch = idx / R, r = idx - ch * R;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
+                    unsigned code = w[u][wi] >> sh;
+                    if (sh + BITS > 32) code |= w[u][wi + 1] << (32 - sh);
+                    X[g.row(ch * 32 + e) + r] = sc[u] * lev[code & MASK];
+                }
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------ the kernel
 
-template <int SIDE, int BT, int PRO, int EPI>
+template <int SIDE, int VW, int NV, int PRO, int EPI>
 __global__ void __launch_bounds__(NT, 1)
-vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const int R) {
+vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const Geo g) {
+    static_assert(NT == 256, "register budget assumes 256 threads");
     extern __shared__ float4 smem_f4[];
     float *X = reinterpret_cast<float *>(smem_f4);
+    constexpr int R = VW * NV;
     const int tid = threadIdx.x;
-    const int d = static_cast<int>(P.d);
-    const int Rp = R;
+    const int d = g.d;
     const int64_t v0 = static_cast<int64_t>(blockIdx.x) * R;
     const int64_t nvec = L.nvec;
     const bool fwd = (L.dir == HARP_FWD);
     const float *__restrict__ signs = P.signs;
+    const int tile_floats = g.row(d - 1) + g.Rp;      // end of the padded tile
 
     // ---------------------------------------------------------- prologue
+    // Every load loop issues IB independent global loads per thread before it
+    // writes any of them to shared memory, so a CTA waits for a few DRAM
+    // round trips rather than one per element.
     if constexpr (PRO == PRO_CODES) {
-        // dequantise R rows of codes into the tile (inverse path)
-        float *lev = X + static_cast<size_t>(d) * Rp;
+        float *lev = X + tile_floats;
         if (tid < 16) lev[tid] = Q.level[tid];
         __syncthreads();
-        const int bits = Q.bits, g = Q.group, ng = d / g;
-        const int64_t rowbytes = static_cast<int64_t>(d) * bits / 8;
-        const unsigned mask = (1u << bits) - 1u;
-        for (int idx = tid; idx < R * d; idx += NT) {
-            const int r = idx / d, i = idx - r * d;
-            const int64_t row = v0 + r;
-            float val = 0.0f;
-            if (row < nvec) {
-                const int64_t bitoff = static_cast<int64_t>(i) * bits;
-                const int64_t byte = bitoff >> 3;
-                const uint8_t *cr = L.in_codes + row * rowbytes;
-                unsigned w = cr[byte];
-                if (byte + 1 < rowbytes) w |= static_cast<unsigned>(cr[byte + 1]) << 8;
-                const int code = static_cast<int>((w >> (bitoff & 7)) & mask);
-                const float s = __half2float(__ushort_as_half(L.in_scales[row * ng + i / g]));
-                val = s * lev[code];
-            }
-            X[i * Rp + r] = val;
-        }
+        if (Q.bits == 2) load_codes<2>(X, g, Q, L, lev, v0, tid);
+        else if (Q.bits == 3) load_codes<3>(X, g, Q, L, lev, v0, tid);
+        else load_codes<4>(X, g, Q, L, lev, v0, tid);
     } else if constexpr (SIDE == SIDE_ROWS) {
-        if ((R & 3) == 0 && (d & 3) == 0) {
+        if (VW == 4 && (d & 3) == 0) {
+            constexpr int IB = 4;
             const int nc4 = d >> 2;
-            for (int idx = tid; idx < (R >> 2) * nc4; idx += NT) {
-                const int rq = idx / nc4, c4 = idx - rq * nc4;
-                float v[4][4];
+            const int n = NV * nc4;
+            for (int base = tid; base < n; base += NT * IB) {
+                float v[IB][4][4];
+                float4 sg[IB];
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    const int64_t row = v0 + rq * 4 + rr;
-                    if (row < nvec) {
-                        ldg4<PRO>(L.in, row * L.ld_in + c4 * 4, v[rr]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) v[rr][e] = 0.0f;
-                    }
-                }
-                if (fwd) {
-                    const float4 sg = __ldg(reinterpret_cast<const float4 *>(signs) + c4);
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    const int c4 = idx / NV, rq = idx - c4 * NV;
+                    sg[u] = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
                     for (int rr = 0; rr < 4; ++rr) {
-                        v[rr][0] *= sg.x; v[rr][1] *= sg.y; v[rr][2] *= sg.z; v[rr][3] *= sg.w;
+                        const int64_t row = v0 + rq * 4 + rr;
+                        if (idx < n && row < nvec) {
+                            ldg4<PRO>(L.in, row * L.ld_in + c4 * 4, v[u][rr]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) v[u][rr][e] = 0.0f;
+                        }
                     }
+                    if (fwd && idx < n) sg[u] = __ldg(reinterpret_cast<const float4 *>(signs) + c4);
                 }
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int e = (p + idx) & 3;
-                    float w[4];
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    if (idx < n) {
+                        const int c4 = idx / NV, rq = idx - c4 * NV;
+                        const float se[4] = {sg[u].x, sg[u].y, sg[u].z, sg[u].w};
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) {
-                        // select v[rr][e] without dynamic register indexing
-                        w[rr] = (e == 0) ? v[rr][0] : (e == 1) ? v[rr][1] : (e == 2) ? v[rr][2] : v[rr][3];
+                        for (int e = 0; e < 4; ++e)
+                            *reinterpret_cast<float4 *>(X + g.row(c4 * 4 + e) + rq * 4) =
+                                make_float4(v[u][0][e] * se[e], v[u][1][e] * se[e], v[u][2][e] * se[e], v[u][3][e] * se[e]);
                     }
-                    *reinterpret_cast<float4 *>(X + (c4 * 4 + e) * Rp + rq * 4) =
-                        make_float4(w[0], w[1], w[2], w[3]);
                 }
             }
         } else {
-            for (int idx = tid; idx < R * d; idx += NT) {
-                const int r = idx / d, i = idx - r * d;
-                const int64_t row = v0 + r;
-                float val = (row < nvec) ? ldg1<PRO>(L.in, row * L.ld_in + i) : 0.0f;
-                if (fwd) val *= __ldg(signs + i);
-                X[i * Rp + r] = val;
+            constexpr int IB = 8;
+            const int n = R * d;
+            for (int base = tid; base < n; base += NT * IB) {
+                float v[IB];
+#pragma unroll
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    const int r = idx / d, i = idx - r * d;
+                    const int64_t row = v0 + r;
+                    v[u] = (idx < n && row < nvec) ? ldg1<PRO>(L.in, row * L.ld_in + i) : 0.0f;
+                    if (fwd && idx < n) v[u] *= __ldg(signs + i);
+                }
+#pragma unroll
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    if (idx < n) {
+                        const int r = idx / d, i = idx - r * d;
+                        X[g.row(i) + r] = v[u];
+                    }
+                }
             }
         }
     } else {  // SIDE_COLS: vectors are columns v0 .. v0+R-1, coordinates are rows
-        if ((R & 3) == 0) {
-            const int nq = R >> 2;
-            for (int idx = tid; idx < d * nq; idx += NT) {
-                const int i = idx / nq, bq = idx - i * nq;
-                const int64_t col = v0 + bq * 4;
-                float v[4];
-                if (col + 3 < nvec) {
-                    ldg4<PRO>(L.in, static_cast<int64_t>(i) * L.ld_in + col, v);
-                } else {
+        if constexpr (VW == 4) {
+            constexpr int IB = 16;
+            const int n = d * NV;
+            for (int base = tid; base < n; base += NT * IB) {
+                float v[IB][4];
+                float sg[IB];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        v[e] = (col + e < nvec) ? ldg1<PRO>(L.in, static_cast<int64_t>(i) * L.ld_in + col + e) : 0.0f;
-                }
-                if (fwd) {
-                    const float sg = __ldg(signs + i);
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    const int i = idx / NV, bq = idx - i * NV;
+                    const int64_t col = v0 + bq * 4;
+                    if (idx < n && col + 3 < nvec) {
+                        ldg4<PRO>(L.in, static_cast<int64_t>(i) * L.ld_in + col, v[u]);
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) v[e] *= sg;
+                        for (int e = 0; e < 4; ++e)
+                            v[u][e] = (idx < n && col + e < nvec)
+                                ? ldg1<PRO>(L.in, static_cast<int64_t>(i) * L.ld_in + col + e) : 0.0f;
+                    }
+                    sg[u] = (fwd && idx < n) ? __ldg(signs + i) : 1.0f;
                 }
-                *reinterpret_cast<float4 *>(X + i * Rp + bq * 4) = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    if (idx < n) {
+                        const int i = idx / NV, bq = idx - i * NV;
+                        *reinterpret_cast<float4 *>(X + g.row(i) + bq * 4) =
+                            make_float4(v[u][0] * sg[u], v[u][1] * sg[u], v[u][2] * sg[u], v[u][3] * sg[u]);
+                    }
+                }
             }
         } else {
-            for (int idx = tid; idx < d * R; idx += NT) {
-                const int i = idx / R, bcol = idx - i * R;
-                const int64_t col = v0 + bcol;
-                float val = (col < nvec) ? ldg1<PRO>(L.in, static_cast<int64_t>(i) * L.ld_in + col) : 0.0f;
-                if (fwd) val *= __ldg(signs + i);
-                X[i * Rp + bcol] = val;
+            constexpr int IB = 8;
+            const int n = d * R;
+            for (int base = tid; base < n; base += NT * IB) {
+                float v[IB];
+#pragma unroll
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    const int i = idx / R, bcol = idx - i * R;
+                    const int64_t col = v0 + bcol;
+                    v[u] = (idx < n && col < nvec) ? ldg1<PRO>(L.in, static_cast<int64_t>(i) * L.ld_in + col) : 0.0f;
+                    if (fwd && idx < n) v[u] *= __ldg(signs + i);
+                }
+#pragma unroll
+                for (int u = 0; u < IB; ++u) {
+                    const int idx = base + u * NT;
+                    if (idx < n) {
+                        const int i = idx / R, bcol = idx - i * R;
+                        X[g.row(i) + bcol] = v[u];
+                    }
+                }
             }
         }
     }
@@ -370,35 +643,22 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const int R) {
     // ---------------------------------------------------------- stages
     for (int ti = 0; ti < P.m; ++ti) {
         const int t = fwd ? ti : P.m - 1 - ti;
-        run_stage<BT>(X, Rp, R, d, P.st[t], L.dir, tid);
+        run_stage<VW, NV>(X, g, P.st[t], t == P.m - 1, L.dir, tid);
     }
 
     // ---------------------------------------------------------- epilogue
     if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
         if constexpr (SIDE == SIDE_ROWS) {
-            if ((R & 3) == 0 && (d & 3) == 0) {
+            if (VW == 4 && (d & 3) == 0) {
                 const int nc4 = d >> 2;
-                for (int idx = tid; idx < (R >> 2) * nc4; idx += NT) {
-                    const int rq = idx / nc4, c4 = idx - rq * nc4;
-                    float v[4][4];  // [row][e]
-                    float sg[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-                    if (!fwd) {
-                        const float4 t4 = __ldg(reinterpret_cast<const float4 *>(signs) + c4);
-                        sg[0] = t4.x; sg[1] = t4.y; sg[2] = t4.z; sg[3] = t4.w;
-                    }
+                for (int idx = tid; idx < NV * nc4; idx += NT) {
+                    const int c4 = idx / NV, rq = idx - c4 * NV;
+                    float v[4][4];   // [row][e]
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const int e = (p + idx) & 3;
-                        const float4 w = *reinterpret_cast<const float4 *>(X + (c4 * 4 + e) * Rp + rq * 4);
-                        const float se = (e == 0) ? sg[0] : (e == 1) ? sg[1] : (e == 2) ? sg[2] : sg[3];
-#pragma unroll
-                        for (int rr = 0; rr < 4; ++rr) {
-                            const float val = ((rr == 0) ? w.x : (rr == 1) ? w.y : (rr == 2) ? w.z : w.w) * se;
-                            if (e == 0) v[rr][0] = val;
-                            else if (e == 1) v[rr][1] = val;
-                            else if (e == 2) v[rr][2] = val;
-                            else v[rr][3] = val;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 w = *reinterpret_cast<const float4 *>(X + g.row(c4 * 4 + e) + rq * 4);
+                        const float se = fwd ? 1.0f : __ldg(signs + c4 * 4 + e);
+                        v[0][e] = w.x * se; v[1][e] = w.y * se; v[2][e] = w.z * se; v[3][e] = w.w * se;
                     }
 #pragma unroll
                     for (int rr = 0; rr < 4; ++rr) {
@@ -410,18 +670,17 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const int R) {
                 for (int idx = tid; idx < R * d; idx += NT) {
                     const int r = idx / d, i = idx - r * d;
                     const int64_t row = v0 + r;
-                    float val = X[i * Rp + r];
+                    float val = X[g.row(i) + r];
                     if (!fwd) val *= __ldg(signs + i);
                     if (row < nvec) stg1<EPI>(L.out, row * L.ld_out + i, val);
                 }
             }
         } else {  // SIDE_COLS
-            if ((R & 3) == 0) {
-                const int nq = R >> 2;
-                for (int idx = tid; idx < d * nq; idx += NT) {
-                    const int i = idx / nq, bq = idx - i * nq;
+            if constexpr (VW == 4) {
+                for (int idx = tid; idx < d * NV; idx += NT) {
+                    const int i = idx / NV, bq = idx - i * NV;
                     const int64_t col = v0 + bq * 4;
-                    const float4 w = *reinterpret_cast<const float4 *>(X + i * Rp + bq * 4);
+                    const float4 w = *reinterpret_cast<const float4 *>(X + g.row(i) + bq * 4);
                     const float sg = fwd ? 1.0f : __ldg(signs + i);
                     float v[4] = {w.x * sg, w.y * sg, w.z * sg, w.w * sg};
                     if (col + 3 < nvec) {
@@ -436,7 +695,7 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const int R) {
                 for (int idx = tid; idx < d * R; idx += NT) {
                     const int i = idx / R, bcol = idx - i * R;
                     const int64_t col = v0 + bcol;
-                    float val = X[i * Rp + bcol];
+                    float val = X[g.row(i) + bcol];
                     if (!fwd) val *= __ldg(signs + i);
                     if (col < nvec) stg1<EPI>(L.out, static_cast<int64_t>(i) * L.ld_out + col, val);
                 }
@@ -444,103 +703,59 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const int R) {
         }
     } else {
         // EPI_QUANT / EPI_QUANT_F32: rows side, forward. g % 32 == 0, g | d.
-        const int g = Q.group, ng = d / g, nchunk = d >> 5, cpg = g >> 5;
-        float *part = X + static_cast<size_t>(d) * Rp;   // [R][nchunk]
-        float *sc = part + R * nchunk;                    // [R][ng]
-        float *thr = sc + R * ng;                         // [16]
-        if (tid < 16) thr[tid] = Q.thr[tid];
-        const bool is_max = (Q.kind == HARP_ABSMAX);
+        const int ng = d / Q.group;
+        float *sc = X + tile_floats;                      // [R][ng] stored scale
+        float *isc = sc + R * ng;                         // [R][ng] its reciprocal
         const int warp = tid >> 5, lane = tid & 31;
-        const int nrv = R / BT;
-        // pass 1: per 32-coordinate chunk statistics
-        for (int item = warp; item < nrv * nchunk; item += NT / 32) {
-            const int rq = item / nchunk, ch = item - rq * nchunk;
-            float x[BT];
-            lds<BT>(X + (ch * 32 + lane) * Rp + rq * BT, x);
-#pragma unroll
-            for (int v = 0; v < BT; ++v) {
-                const float st = warp_reduce(is_max ? fabsf(x[v]) : x[v] * x[v], is_max);
-                if (lane == 0) part[(rq * BT + v) * nchunk + ch] = st;
-            }
-        }
-        __syncthreads();
-        // pass 2: group scales (combined in chunk order)
-        for (int idx = tid; idx < R * ng; idx += NT) {
-            const int r = idx / ng, gi = idx - r * ng;
-            float stat = 0.0f;
-            for (int c = 0; c < cpg; ++c) {
-                const float p = part[r * nchunk + gi * cpg + c];
-                stat = is_max ? fmaxf(stat, p) : stat + p;
-            }
-            const unsigned short hb = group_scale_bits(stat, Q);
-            sc[idx] = __half2float(__ushort_as_half(hb));
-            const int64_t row = v0 + r;
-            if (row < nvec) L.scales[row * ng + gi] = hb;
-        }
-        __syncthreads();
-        // pass 3: codes, packing (and the optional fp32 copy of the rotated rows)
-        const int bits = Q.bits;
-        const int64_t rowbytes = static_cast<int64_t>(d) * bits / 8;
-        for (int item = warp; item < nrv * nchunk; item += NT / 32) {
-            const int rq = item / nchunk, ch = item - rq * nchunk;
-            const int i = ch * 32 + lane;
-            const int gi = (ch * 32) / g;
-            float x[BT];
-            lds<BT>(X + i * Rp + rq * BT, x);
-#pragma unroll
-            for (int v = 0; v < BT; ++v) {
-                const int r = rq * BT + v;
-                const int64_t row = v0 + r;
-                const int code = quant_code(x[v], sc[r * ng + gi], Q, thr);
-                const unsigned word = pack_warp(code, bits, lane);
-                if (row < nvec) {
-                    if (lane < bits)
-                        reinterpret_cast<unsigned *>(L.codes + row * rowbytes)[ch * bits + lane] = word;
-                    if constexpr (EPI == EPI_QUANT_F32)
-                        static_cast<float *>(L.out)[row * L.ld_out + i] = x[v];
-                }
-            }
-        }
+        constexpr bool F32OUT = (EPI == EPI_QUANT_F32);
+        if (Q.bits == 2) quantize_tile<VW, 2, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
+        else if (Q.bits == 3) quantize_tile<VW, 3, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
+        else quantize_tile<VW, 4, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
     }
 }
 
 // ------------------------------------------------------------ standalone codec
 
-// One warp per (row, group): statistics chunk by chunk in the same order as
-// the fused epilogue, then codes and packing.
-template <int PRO>
+// One warp per (row, group): statistics in the same order as the fused
+// epilogue (per-lane accumulation, then the xor tree), then codes and packing.
+template <int PRO, int BITS>
+__device__ __forceinline__ void quantize_group(const QuantDev &Q, const void *in, int64_t off,
+                                               uint8_t *codes_row, uint16_t *scale, int64_t word0,
+                                               int lane, const float (&t)[(1 << BITS) - 1]) {
+    const int gsz = Q.group;
+    const bool is_max = (Q.kind == HARP_ABSMAX);
+    float st = 0.0f;
+    for (int c = 0; c < (gsz >> 5); ++c) st = combine(st, ldg1<PRO>(in, off + c * 32 + lane), is_max);
+    st = warp_reduce(st, is_max);
+    const unsigned short hb = group_scale_bits(st, Q);
+    if (lane == 0) *scale = hb;
+    const float s = __half2float(__ushort_as_half(hb));
+    const float is = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+    for (int c = 0; c < (gsz >> 5); ++c) {
+        const float x = ldg1<PRO>(in, off + c * 32 + lane);
+        const int code = code_of<BITS>(x, s, is, !is_max, t);
+        const unsigned word = pack_words<BITS>(code, lane);
+        if (lane < BITS) reinterpret_cast<unsigned *>(codes_row)[word0 + c * BITS + lane] = word;
+    }
+}
+
+template <int PRO, int BITS>
 __global__ void __launch_bounds__(256)
 quantize_kernel(const QuantDev Q, const void *in, int64_t rows, int64_t cols, int64_t ld_in,
                 uint8_t *codes, uint16_t *scales) {
-    __shared__ float thr[16];
-    if (threadIdx.x < 16) thr[threadIdx.x] = Q.thr[threadIdx.x];
-    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    const int g = Q.group, bits = Q.bits;
+    const int g = Q.group;
     const int64_t ng = cols / g;
-    const int64_t rowbytes = cols * bits / 8;
-    const bool is_max = (Q.kind == HARP_ABSMAX);
+    const int64_t rowbytes = cols * BITS / 8;
+    float t[(1 << BITS) - 1];
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) t[k] = Q.thr[k];
     for (int64_t item = warp; item < rows * ng; item += nwarps) {
         const int64_t row = item / ng, gi = item - row * ng;
-        const int64_t off = row * ld_in + gi * g;
-        float stat = 0.0f;
-        for (int c = 0; c < (g >> 5); ++c) {
-            const float x = ldg1<PRO>(in, off + c * 32 + lane);
-            const float p = warp_reduce(is_max ? fabsf(x) : x * x, is_max);
-            stat = is_max ? fmaxf(stat, p) : stat + p;
-        }
-        const unsigned short hb = group_scale_bits(stat, Q);
-        if (lane == 0) scales[row * ng + gi] = hb;
-        const float s = __half2float(__ushort_as_half(hb));
-        for (int c = 0; c < (g >> 5); ++c) {
-            const float x = ldg1<PRO>(in, off + c * 32 + lane);
-            const int code = quant_code(x, s, Q, thr);
-            const unsigned word = pack_warp(code, bits, lane);
-            if (lane < bits)
-                reinterpret_cast<unsigned *>(codes + row * rowbytes)[((gi * g) >> 5) * bits + c * bits + lane] = word;
-        }
+        quantize_group<PRO, BITS>(Q, in, row * ld_in + gi * g, codes + row * rowbytes, scales + row * ng + gi,
+                                  ((gi * g) >> 5) * BITS, lane, t);
     }
 }
 
@@ -567,91 +782,116 @@ dequantize_kernel(const QuantDev Q, const uint8_t *codes, const uint16_t *scales
 
 // ------------------------------------------------------------ host dispatch
 
-int extra_smem_floats(int R, int d, int epi, int pro, int group) {
-    int extra = 0;
-    if (epi == EPI_QUANT || epi == EPI_QUANT_F32) extra += R * (d / 32) + R * (d / group) + 16;
-    if (pro == PRO_CODES) extra += 16;
-    return extra;
+struct TileChoice {
+    int R, VW, NV;
+};
+
+// Tile heights the kernels are built for: 4*NV vectors (NV = 1, 2, 3, 8) and
+// the narrow 1- and 2-vector tiles for very long vectors.
+constexpr TileChoice kTiles[] = {{32, 4, 8}, {12, 4, 3}, {8, 4, 2}, {4, 4, 1}, {2, 2, 1}, {1, 1, 1}};
+
+int last_radix(const PlanDev &plan) { return plan.st[plan.m - 1].b; }
+
+Geo make_geo(const PlanDev &plan, const TileChoice &t) {
+    Geo g{};
+    g.d = static_cast<int>(plan.d);
+    g.R = t.R;
+    g.Rp = t.R;
+    g.padq = t.VW;
+    g.bl = last_radix(plan);
+    g.bl_shift = (g.bl & (g.bl - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(g.bl)) : -1;
+    return g;
 }
 
-int pick_tile(int64_t d, int epi, int pro, int group) {
-    static const int cand[] = {32, 28, 24, 20, 16, 12, 8, 6, 4, 2, 1};
-    for (int R : cand) {
-        const int64_t floats = d * R + extra_smem_floats(R, static_cast<int>(d), epi, pro, group);
-        if (floats * 4 <= SMEM_MAX) return R;
-    }
-    return 0;
+int64_t smem_floats(const PlanDev &plan, const TileChoice &t, int epi, int pro, int group) {
+    const int64_t d = plan.d;
+    const int bl = last_radix(plan);
+    int64_t f = d * t.R + static_cast<int64_t>(t.VW) * ((d - 1) / bl);
+    if (epi == EPI_QUANT || epi == EPI_QUANT_F32) f += 2 * t.R * (d / group);
+    if (pro == PRO_CODES) f += 16;
+    return f;
 }
 
-using KernelFn = void (*)(const PlanDev, const QuantDev, const VecLaunch, const int);
+int pick_tile(const PlanDev &plan, int epi, int pro, int group) {
+    for (int i = 0; i < static_cast<int>(sizeof(kTiles) / sizeof(kTiles[0])); ++i)
+        if (smem_floats(plan, kTiles[i], epi, pro, group) * 4 <= SMEM_MAX) return i;
+    return -1;
+}
 
-template <int SIDE, int BT, int PRO, int EPI>
+using KernelFn = void (*)(const PlanDev, const QuantDev, const VecLaunch, const Geo);
+
+template <int SIDE, int VW, int NV, int PRO, int EPI>
 KernelFn get_kernel() {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(vec_kernel<SIDE, BT, PRO, EPI>,
+        attr_err = cudaFuncSetAttribute(vec_kernel<SIDE, VW, NV, PRO, EPI>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAX);
     });
-    return attr_err == cudaSuccess ? vec_kernel<SIDE, BT, PRO, EPI> : nullptr;
+    return attr_err == cudaSuccess ? vec_kernel<SIDE, VW, NV, PRO, EPI> : nullptr;
 }
 
-template <int SIDE, int BT>
+template <int SIDE, int VW, int NV>
 KernelFn select_pe(int pro, int epi) {
     if constexpr (SIDE == SIDE_ROWS) {
         if (pro == PRO_CODES) {
-            if (epi == EPI_F32) return get_kernel<SIDE, BT, PRO_CODES, EPI_F32>();
-            if (epi == EPI_BF16) return get_kernel<SIDE, BT, PRO_CODES, EPI_BF16>();
+            if (epi == EPI_F32) return get_kernel<SIDE, VW, NV, PRO_CODES, EPI_F32>();
+            if (epi == EPI_BF16) return get_kernel<SIDE, VW, NV, PRO_CODES, EPI_BF16>();
             return nullptr;
         }
-#define HARP_ROW_CASE(P)                                                          \
-    if (pro == P) {                                                               \
-        if (epi == EPI_F32) return get_kernel<SIDE, BT, P, EPI_F32>();            \
-        if (epi == EPI_BF16) return get_kernel<SIDE, BT, P, EPI_BF16>();          \
-        if (epi == EPI_QUANT) return get_kernel<SIDE, BT, P, EPI_QUANT>();        \
-        if (epi == EPI_QUANT_F32) return get_kernel<SIDE, BT, P, EPI_QUANT_F32>(); \
+#define HARP_ROW_CASE(P)                                                              \
+    if (pro == P) {                                                                   \
+        if (epi == EPI_F32) return get_kernel<SIDE, VW, NV, P, EPI_F32>();            \
+        if (epi == EPI_BF16) return get_kernel<SIDE, VW, NV, P, EPI_BF16>();          \
+        if (epi == EPI_QUANT) return get_kernel<SIDE, VW, NV, P, EPI_QUANT>();        \
+        if (epi == EPI_QUANT_F32) return get_kernel<SIDE, VW, NV, P, EPI_QUANT_F32>(); \
     }
         HARP_ROW_CASE(PRO_F32)
         HARP_ROW_CASE(PRO_BF16)
 #undef HARP_ROW_CASE
         return nullptr;
     } else {
-        if (pro == PRO_F32 && epi == EPI_F32) return get_kernel<SIDE, BT, PRO_F32, EPI_F32>();
-        if (pro == PRO_F32 && epi == EPI_BF16) return get_kernel<SIDE, BT, PRO_F32, EPI_BF16>();
-        if (pro == PRO_BF16 && epi == EPI_F32) return get_kernel<SIDE, BT, PRO_BF16, EPI_F32>();
-        if (pro == PRO_BF16 && epi == EPI_BF16) return get_kernel<SIDE, BT, PRO_BF16, EPI_BF16>();
+        if (pro == PRO_F32 && epi == EPI_F32) return get_kernel<SIDE, VW, NV, PRO_F32, EPI_F32>();
+        if (pro == PRO_F32 && epi == EPI_BF16) return get_kernel<SIDE, VW, NV, PRO_F32, EPI_BF16>();
+        if (pro == PRO_BF16 && epi == EPI_F32) return get_kernel<SIDE, VW, NV, PRO_BF16, EPI_F32>();
+        if (pro == PRO_BF16 && epi == EPI_BF16) return get_kernel<SIDE, VW, NV, PRO_BF16, EPI_BF16>();
         return nullptr;
     }
 }
 
 template <int SIDE>
-KernelFn select_bt(int bt, int pro, int epi) {
-    if (bt == 4) return select_pe<SIDE, 4>(pro, epi);
-    if (bt == 2) return select_pe<SIDE, 2>(pro, epi);
-    return select_pe<SIDE, 1>(pro, epi);
+KernelFn select_tile(int ti, int pro, int epi) {
+    switch (ti) {
+        case 0: return select_pe<SIDE, 4, 8>(pro, epi);
+        case 1: return select_pe<SIDE, 4, 3>(pro, epi);
+        case 2: return select_pe<SIDE, 4, 2>(pro, epi);
+        case 3: return select_pe<SIDE, 4, 1>(pro, epi);
+        case 4: return select_pe<SIDE, 2, 1>(pro, epi);
+        default: return select_pe<SIDE, 1, 1>(pro, epi);
+    }
 }
 
 }  // namespace
 
-int vec_tile(int64_t d, int epi, int group) {
-    return pick_tile(d, epi, PRO_F32, group > 0 ? group : 32);
+int vec_tile(const PlanDev &plan, int epi, int group) {
+    const int ti = pick_tile(plan, epi, PRO_F32, group > 0 ? group : 32);
+    return ti < 0 ? 0 : kTiles[ti].R;
 }
 
 int launch_vec(const PlanDev &plan, const QuantDev *q, const VecLaunch &L, void *stream) {
     const int group = q ? q->group : 32;
-    const int R = pick_tile(plan.d, L.epi, L.pro, group);
-    if (R == 0) return static_cast<int>(cudaErrorInvalidValue);
-    const int bt = (R % 4 == 0) ? 4 : (R % 2 == 0) ? 2 : 1;
-    KernelFn fn = (L.side == HARP_RIGHT) ? select_bt<SIDE_ROWS>(bt, L.pro, L.epi)
-                                         : select_bt<SIDE_COLS>(bt, L.pro, L.epi);
+    const int ti = pick_tile(plan, L.epi, L.pro, group);
+    if (ti < 0) return static_cast<int>(cudaErrorInvalidValue);
+    KernelFn fn = (L.side == HARP_RIGHT) ? select_tile<SIDE_ROWS>(ti, L.pro, L.epi)
+                                         : select_tile<SIDE_COLS>(ti, L.pro, L.epi);
     if (!fn) return static_cast<int>(cudaErrorInvalidDeviceFunction);
     if (L.nvec == 0) return 0;
-    const int64_t grid = (L.nvec + R - 1) / R;
-    const size_t smem = static_cast<size_t>(plan.d * R +
-        extra_smem_floats(R, static_cast<int>(plan.d), L.epi, L.pro, group)) * 4;
+    const TileChoice &t = kTiles[ti];
+    const int64_t grid = (L.nvec + t.R - 1) / t.R;
+    const size_t smem = static_cast<size_t>(smem_floats(plan, t, L.epi, L.pro, group)) * 4;
     QuantDev qd{};
     if (q) qd = *q;
-    fn<<<static_cast<unsigned>(grid), NT, smem, static_cast<cudaStream_t>(stream)>>>(plan, qd, L, R);
+    fn<<<static_cast<unsigned>(grid), NT, smem, static_cast<cudaStream_t>(stream)>>>(plan, qd, L, make_geo(plan, t));
     return static_cast<int>(cudaGetLastError());
 }
 
@@ -662,10 +902,18 @@ int launch_quantize(const QuantDev &q, const void *in, int in_dtype, int64_t row
     int64_t blocks = (items + 7) / 8;          // 8 warps per block
     if (blocks > 148 * 16) blocks = 148 * 16;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (in_dtype == HARP_F32)
-        quantize_kernel<PRO_F32><<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, in, rows, cols, ld_in, codes, scales);
-    else
-        quantize_kernel<PRO_BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, in, rows, cols, ld_in, codes, scales);
+    const unsigned nb = static_cast<unsigned>(blocks);
+#define HARP_QLAUNCH(P, B) quantize_kernel<P, B><<<nb, 256, 0, st>>>(q, in, rows, cols, ld_in, codes, scales)
+    if (in_dtype == HARP_F32) {
+        if (q.bits == 2) HARP_QLAUNCH(PRO_F32, 2);
+        else if (q.bits == 3) HARP_QLAUNCH(PRO_F32, 3);
+        else HARP_QLAUNCH(PRO_F32, 4);
+    } else {
+        if (q.bits == 2) HARP_QLAUNCH(PRO_BF16, 2);
+        else if (q.bits == 3) HARP_QLAUNCH(PRO_BF16, 3);
+        else HARP_QLAUNCH(PRO_BF16, 4);
+    }
+#undef HARP_QLAUNCH
     return static_cast<int>(cudaGetLastError());
 }
 
