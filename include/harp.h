@@ -229,6 +229,45 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
                              int64_t cols, void *out, int out_dtype, void *workspace,
                              size_t ws_bytes, void *stream);
 
+/* ------------------------------------------- variant that allocates nothing */
+
+/* Capacity of the library-owned scratch used by harp_rotate_quantize_static:
+ * 32 MiB, i.e. a two-sided matrix of up to 8,388,608 elements (for example
+ * 2048 x 4096). */
+#define HARP_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+/* harp_rotate_quantize without a caller workspace. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory: code hosted by a framework that owns every device byte (a pool
+ * reserved at start-up that rejects further requests) and code on a
+ * latency-critical path where cudaMalloc, which may synchronise the device,
+ * is not allowed. Such callers still pass their own input and outputs.
+ *
+ * Arguments and results are those of harp_rotate_quantize (same checks, same
+ * kernels, identical output); the fp32 intermediate of the two-sided path
+ * lives instead in a file-scope device array of HARP_STATIC_WORKSPACE_BYTES
+ * inside the library, which every device that loads the library holds until
+ * the process exits. The call allocates no memory (no cudaMalloc / cudaFree,
+ * no allocating library routine).
+ *  - Size limit: rows*cols*4 bytes (harp_workspace_size) above
+ *    HARP_STATIC_WORKSPACE_BYTES returns HARP_ERR_WORKSPACE before anything
+ *    is launched. Right-only calls (left = NULL) need no scratch.
+ *  - Set-up: the first two-sided call on a device looks up the array's
+ *    device address (cudaGetSymbolAddress, with that device current) and
+ *    caches it; make that first call before any stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    last call's contents. Each call overwrites every element it reads
+ *    before reading it, so nothing needs clearing, but calls that can
+ *    overlap on the GPU (different streams, no ordering between them) race
+ *    on the array and corrupt each other's results: serialise them.
+ * Errors: those of harp_rotate_quantize, plus HARP_ERR_WORKSPACE (too large),
+ * HARP_ERR_CUDA (no device, address lookup failed) and HARP_ERR_UNSUPPORTED
+ * (device ordinal above 63). */
+int harp_rotate_quantize_static(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,
+                                const void *in, int in_dtype, int64_t rows, int64_t cols,
+                                uint8_t *codes, uint16_t *scales, float *rotated_out,
+                                void *stream);
+
 #ifdef __cplusplus
 }
 #endif

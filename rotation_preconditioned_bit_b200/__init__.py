@@ -26,6 +26,7 @@ HARP_FWD, HARP_INV = 0, 1
 HARP_LLOYD_MAX, HARP_ABSMAX = 0, 1
 HARP_BLOCKS_HADAMARD, HARP_BLOCKS_QR, HARP_BLOCKS_CAYLEY = 0, 1, 2
 HARP_MAX_STAGES = 16
+HARP_STATIC_WORKSPACE_BYTES = 32 << 20
 
 BLOCK_KINDS = {"hadamard": HARP_BLOCKS_HADAMARD, "qr": HARP_BLOCKS_QR,
                "cayley_hadamard": HARP_BLOCKS_CAYLEY}
@@ -37,7 +38,7 @@ EXPORTS = (
     "harp_plan_info", "harp_stage_blocks", "harp_lloyd_max_centroids",
     "harp_codebook_create", "harp_codebook_destroy", "harp_codebook_tables",
     "harp_workspace_size", "harp_rotate", "harp_quantize", "harp_dequantize",
-    "harp_rotate_quantize", "harp_dequantize_unrotate",
+    "harp_rotate_quantize", "harp_dequantize_unrotate", "harp_rotate_quantize_static",
 )
 
 
@@ -81,6 +82,7 @@ def lib():
                                            ctypes.c_size_t, _P]
         L.harp_dequantize_unrotate.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _P, _INT, _P,
                                                ctypes.c_size_t, _P]
+        L.harp_rotate_quantize_static.argtypes = [_P, _P, _P, _P, _INT, _I64, _I64, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -263,6 +265,20 @@ def harp_rotate_quantize(left, right, cb, x, codes, scales, rotated_out=None, wo
                                       _ptr(x), _dtype_code(x), rows, cols, _ptr(codes), _ptr(scales),
                                       _ptr(rotated_out), _ptr(workspace), ws, _stream(stream)),
            "harp_rotate_quantize")
+    return codes, scales
+
+
+def harp_rotate_quantize_static(left, right, cb, x, codes, scales, rotated_out=None, stream=None):
+    """harp_rotate_quantize with the two-sided intermediate in the library's
+    own device array (HARP_STATIC_WORKSPACE_BYTES): for callers that cannot
+    allocate device memory. Calls on one device share that array; do not
+    overlap them on the GPU."""
+    _require_cuda(x, codes, scales, rotated_out)
+    rows, cols = x.shape
+    _check(lib().harp_rotate_quantize_static(left.handle if left else None, right.handle, cb.handle,
+                                             _ptr(x), _dtype_code(x), rows, cols, _ptr(codes),
+                                             _ptr(scales), _ptr(rotated_out), _stream(stream)),
+           "harp_rotate_quantize_static")
     return codes, scales
 
 

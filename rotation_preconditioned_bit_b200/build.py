@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libharp.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("harp_kernels.cu", "harp_api.cpp")]
+SOURCES = [os.path.join(CSRC, f) for f in ("harp_kernels.cu", "harp_api.cpp", "harp_static_ws.cu")]
 HEADERS = [os.path.join(CSRC, "harp_internal.h"), os.path.join(INCLUDE, "harp.h")]
 CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
