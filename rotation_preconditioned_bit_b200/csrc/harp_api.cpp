@@ -36,6 +36,10 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 int cuda_status(int err) { return err == 0 ? HARP_OK : HARP_ERR_CUDA; }
 
+// Padded block shape of the pass kernels (see StageDev).
+int pass_jpad(int b) { return (b + 3) & ~3; }
+int pass_kp(int b) { return b <= 8 ? 8 : (b + 15) & ~15; }
+
 // ------------------------------------------------------------ block makers
 // HARP (gist.science paper 2605.29843) section 2.2: B = Q(theta) G_b.
 
@@ -265,11 +269,16 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
     // host staging of the device layout
     const size_t sign_floats = (static_cast<size_t>(d) + 3) & ~static_cast<size_t>(3);
     size_t total = sign_floats;
-    std::vector<size_t> off(m);
+    std::vector<size_t> off(m), poff(m);
     for (int t = 0; t < m; ++t) {
         const int kpad = (radix[t] + 3) & ~3;
         off[t] = total;
         total += 2 * static_cast<size_t>(d) * kpad;   // fwd then inv
+    }
+    for (int t = 0; t < m; ++t) {                       // pass-kernel layout
+        const int b = radix[t];
+        poff[t] = total;
+        total += 2 * static_cast<size_t>(d / b) * pass_jpad(b) * pass_kp(b);
     }
     std::vector<float> host;
     try { host.assign(total, 0.0f); } catch (...) { return HARP_ERR_ALLOC; }
@@ -285,6 +294,17 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
                 for (int j = 0; j < b; ++j) {
                     fwd[(c * b + j) * kpad + k] = B[k * b + j];
                     inv[(c * b + k) * kpad + j] = B[k * b + j];
+                }
+        }
+        const int jp = pass_jpad(b), kp = pass_kp(b);
+        float *pf = host.data() + poff[t];
+        float *pi = pf + static_cast<size_t>(ng) * jp * kp;
+        for (int64_t c = 0; c < ng; ++c) {
+            const float *B = blocks[t] + c * b * b;
+            for (int j = 0; j < b; ++j)
+                for (int k = 0; k < b; ++k) {
+                    pf[(c * jp + j) * kp + k] = B[k * b + j];
+                    pi[(c * jp + j) * kp + k] = B[j * b + k];
                 }
         }
     }
@@ -318,6 +338,10 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
         p->dev.st[t].s = s;
         p->dev.st[t].fwd = base + off[t];
         p->dev.st[t].inv = base + off[t] + static_cast<size_t>(d) * kpad;
+        p->dev.st[t].jpad = pass_jpad(b);
+        p->dev.st[t].kp = pass_kp(b);
+        p->dev.st[t].pfwd = base + poff[t];
+        p->dev.st[t].pinv = base + poff[t] + static_cast<size_t>(d / b) * pass_jpad(b) * pass_kp(b);
     }
     *out = p;
     return HARP_OK;
@@ -465,7 +489,9 @@ static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, i
     if (st) return st;
     if (right->d != cols) return HARP_ERR_SHAPE;
     if (left && left->d != rows) return HARP_ERR_SHAPE;
-    if (harp::vec_tile(right->dev, harp::EPI_QUANT, cb->q.group) == 0) return HARP_ERR_UNSUPPORTED;
+    if (!(left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group)) &&
+        harp::vec_tile(right->dev, harp::EPI_QUANT, cb->q.group) == 0)
+        return HARP_ERR_UNSUPPORTED;
     if (left) {
         const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(cols) * 4;
         if (need && (!workspace || ws_bytes < need)) return HARP_ERR_WORKSPACE;
@@ -486,6 +512,9 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
     if (!aligned(in, 16) || !aligned(codes, 4) || !aligned(scales, 2) ||
         (rotated_out && !aligned(rotated_out, 16)) || cols % 4)
         return HARP_ERR_ALIGNMENT;
+    if (left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group))
+        return cuda_status(harp::launch_pass_fwd(left->dev, right->dev, cb->q, in, in_dtype, codes, scales,
+                                                 rotated_out, static_cast<float *>(workspace), stream));
     const int pro_in = (in_dtype == HARP_F32) ? harp::PRO_F32 : harp::PRO_BF16;
     const void *row_in = in;
     int row_pro = pro_in;
@@ -530,6 +559,9 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
     if (rows == 0 || cols == 0) return HARP_OK;
     if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
     if (!aligned(out, 16) || !aligned(scales, 2) || cols % 4) return HARP_ERR_ALIGNMENT;
+    if (left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group))
+        return cuda_status(harp::launch_pass_inv(left->dev, right->dev, cb->q, codes, scales, out, out_dtype,
+                                                 static_cast<float *>(workspace), stream));
     harp::VecLaunch Lr{};
     Lr.side = HARP_RIGHT;
     Lr.dir = HARP_INV;

@@ -21,6 +21,14 @@ struct StageDev {
     int64_t s;
     const float *fwd;
     const float *inv;
+    // The same blocks for the pass kernels, [d/b][jpad][kp] floats with
+    // jpad = b rounded up to 4 and kp = b rounded up to 8 (b <= 8) or 16:
+    //   pfwd[c][j][k] = B_{t,c}[k][j],  pinv[c][j][k] = B_{t,c}[j][k]
+    // (coefficient of input j in output k), zero in the padding.
+    int jpad;
+    int kp;
+    const float *pfwd;
+    const float *pinv;
 };
 
 struct PlanDev {
@@ -68,6 +76,19 @@ int launch_quantize(const QuantDev &q, const void *in, int in_dtype, int64_t row
 int launch_dequantize(const QuantDev &q, const uint8_t *codes, const uint16_t *scales,
                       int64_t rows, int64_t cols, void *out, int out_dtype, int64_t ld_out,
                       void *stream);
+
+// Pass kernels (harp_pass.cu): the two-sided paths as a short sequence of
+// tiled passes over the matrix, each applying a run of stages of both
+// processors to a digit-box tile held in shared memory. `ws` is an fp32
+// rows x cols workspace; every pass updates its tiles in place.
+// pass_plan_ok: whether such a plan exists for these processors and group.
+bool pass_plan_ok(const PlanDev &left, const PlanDev &right, int group);
+int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q, const void *in,
+                    int in_dtype, uint8_t *codes, uint16_t *scales, float *rotated_out, float *ws,
+                    void *stream);
+int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q,
+                    const uint8_t *codes, const uint16_t *scales, void *out, int out_dtype,
+                    float *ws, void *stream);
 
 // Vectors per CTA the whole-vector kernel uses for this plan and epilogue
 // (0 if a vector does not fit in shared memory).

@@ -1,0 +1,104 @@
+// harp_quant_dev.cuh -- device helpers of the group quantizer shared by the
+// kernels of libharp: PolarQuant (gist.science paper 2603.29078) section 2
+// (RMS group scale to N(0,1), Lloyd-Max code, fp16 scale) and section 1
+// (absmax uniform code), plus the LSB-first bit packing of the codes.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "harp_internal.h"
+
+namespace harp {
+namespace dq {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// Warp-wide reduction (xor butterfly, fixed order): sum or max.
+__device__ __forceinline__ float warp_reduce(float v, bool is_max) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const float w = __shfl_xor_sync(FULL, v, o);
+        v = is_max ? fmaxf(v, w) : v + w;
+    }
+    return v;
+}
+
+// Group scale from the combined statistic: RMS (Lloyd-Max) or absmax/qmax,
+// rounded to fp16 (nearest even), saturating at 65504.
+__device__ __forceinline__ unsigned short group_scale_bits(float stat, const QuantDev &Q) {
+    float s;
+    if (Q.kind == HARP_LLOYD_MAX) {
+        s = sqrtf(stat / static_cast<float>(Q.group));
+    } else {
+        s = stat / static_cast<float>((1 << (Q.bits - 1)) - 1);
+    }
+    s = fminf(s, 65504.0f);
+    return __half_as_ushort(__float2half_rn(s));
+}
+
+
+// ------------------------------------------------------------ codes
+
+// t[OFF + STRIDE * idx] for idx in [0, N) (N a power of two) by a tree of
+// selects on the bits of idx: the array stays in registers.
+template <int OFF, int N, int STRIDE, int K>
+__device__ __forceinline__ float pick(const float (&t)[K], int idx) {
+    if constexpr (N == 1) {
+        return t[OFF];
+    } else {
+        return (idx & (N / 2)) ? pick<OFF + STRIDE * (N / 2), N / 2, STRIDE, K>(t, idx)
+                               : pick<OFF, N / 2, STRIDE, K>(t, idx);
+    }
+}
+
+// Lloyd-Max code = number of midpoints below z: binary search over the
+// sorted fp32 midpoints held in registers (ties go to the lower code).
+template <int BITS, int STEP = (1 << (BITS - 1))>
+__device__ __forceinline__ int lm_search(float z, const float (&t)[(1 << BITS) - 1], int code) {
+    if constexpr (STEP == 0) {
+        return code;
+    } else {
+        constexpr int K = 1 << BITS;
+        const float th = pick<STEP - 1, K / (2 * STEP), 2 * STEP, K - 1>(t, code / (2 * STEP));
+        return lm_search<BITS, STEP / 2>(z, t, code + ((z > th) ? STEP : 0));
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ int code_of(float x, float s, float inv_s, bool lloyd,
+                                       const float (&t)[(1 << BITS) - 1]) {
+    constexpr int HALF = 1 << (BITS - 1);
+    if (!(s > 0.0f)) return HALF;
+    const float z = x * inv_s;
+    if (lloyd) return lm_search<BITS>(z, t, 0);
+    const float qmax = static_cast<float>(HALF - 1);
+    return static_cast<int>(fminf(fmaxf(rintf(z), -qmax), qmax)) + HALF;
+}
+
+template <int BITS>
+__device__ __forceinline__ unsigned pack_words(int code, int lane) {
+    const int bit0 = BITS * lane;
+    const int wlo = bit0 >> 5, sh = bit0 & 31;
+    const unsigned lo = static_cast<unsigned>(code) << sh;
+    const unsigned hi = (sh + BITS > 32) ? (static_cast<unsigned>(code) >> (32 - sh)) : 0u;
+    unsigned mine = 0;
+#pragma unroll
+    for (int w = 0; w < BITS; ++w) {
+        const unsigned part = (w == wlo ? lo : 0u) | (w == wlo + 1 ? hi : 0u);
+        const unsigned word = __reduce_or_sync(FULL, part);
+        if (w == lane) mine = word;
+    }
+    return mine;
+}
+
+// Group statistic of `g` consecutive values for one vector: each lane
+// accumulates its values (coordinates lane, lane+32, ...) in order, then a
+// fixed xor tree combines the lanes. The standalone quantizer uses the same
+// order, so both give identical scales.
+__device__ __forceinline__ float combine(float a, float x, bool is_max) {
+    return is_max ? fmaxf(a, fabsf(x)) : fmaf(x, x, a);
+}
+
+
+}  // namespace dq
+}  // namespace harp

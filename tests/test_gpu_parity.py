@@ -101,9 +101,15 @@ def test_c2_two_sided_full_matrix(c2_ref, qi):
     assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
 
 
-def test_c2_unfused_equals_fused(c2_ref):
-    w, _ = c2_ref
+def test_c2_unfused_matches_oracle_like_fused(c2_ref):
+    """The separate calls (left rotation, right rotation, standalone
+    quantizer) meet the same bar against the oracle as the fused call. The
+    two paths run different kernels that sum in different orders, so their
+    codes may differ only inside the boundary band, which compare_quant
+    excludes and counts."""
+    w, ref = c2_ref
     q = w.quants[1]
+    oc, osc, m, sm = oracle.quantize(q.kind, q.bits, q.group, ref)
     left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
     cb = harp.Codebook(q.kind, q.bits, q.group)
     x = to_dev(w)
@@ -112,9 +118,11 @@ def test_c2_unfused_equals_fused(c2_ref):
     harp.harp_rotate(left, harp.HARP_LEFT, harp.HARP_FWD, x, t)
     t2 = torch.empty_like(t)
     harp.harp_rotate(right, harp.HARP_RIGHT, harp.HARP_FWD, t, t2)
+    assert rel_l2(t2.cpu().numpy(), ref) <= TOL_F32
     c2, s2 = harp.empty_codes(*x.shape, cb)
     harp.harp_quantize(cb, t2, c2, s2)
-    assert torch.equal(c2, codes) and torch.equal(s2, scales)
+    compare_quant(c2.cpu().numpy(), scales_np(s2), oc, osc, m, sm, q.bits, q.group)
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, q.bits, q.group)
 
 
 # ------------------------------------------------------------ [T, 4096] activations, per-token absmax
