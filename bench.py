@@ -6,14 +6,15 @@ nu = 3 entries x 0.02, 0.5 % of input channels x 20), two-sided processor
 (16,16,16) x (16,16,16) with random orthogonal blocks and random signs,
 Lloyd-Max N(0,1) codebooks with group 128 at 2 and at 4 bits.
 
-One step = the whole hot path over that weight, for each bit width:
-rotate + quantize + pack (column kernel, then fused row kernel), then
-dequantize + unrotate (row kernel, then column kernel): 8 kernel launches.
+One step = the whole hot path over that weight, for each bit width, through
+the public two-sided calls: harp_rotate_quantize (rotate both sides,
+quantize, pack) then harp_dequantize_unrotate (decode, inverse rotation, bf16
+out). Each call runs the library's pass kernels (two for this plan), which
+bench.py times one by one with events the library records between them.
 value = algorithmic bytes of the step (bf16 weight read and codes + fp16
 scales written by each forward; codes + scales read and the bf16 weight
 written by each inverse) / device time, in GB/s. The fp32 intermediate
-between the column and row passes is implementation traffic and is not
-credited. L2 is flushed (512 MB write) before every timed step.
+between the passes is implementation traffic and is not credited. L2 is flushed (512 MB write) before every timed step.
 
 --impl reference times the float64 oracle (the CPU statement of the same
 computation) on the host cores instead, on a bounded sample of the same
@@ -156,37 +157,46 @@ def run_gpu(args, rank, world, local_rank):
     cbs = [harp.Codebook("lloyd_max", b, GROUP) for b in BITS]
     x_host = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
     x = x_host.to(dev)
-    ws = torch.empty((ROWS, COLS), dtype=torch.float32, device=dev)
+    ws = harp.empty_workspace(left, right, ROWS, COLS, dev)
     out = torch.empty((ROWS, COLS), dtype=torch.bfloat16, device=dev)
     outs = [harp.empty_codes(ROWS, COLS, cb, dev) for cb in cbs]
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    # one step through the single-kernel entry points, events between launches
-    # (the same four kernels the two-sided calls launch, in the same order)
-    names = ["col_fwd", "row_fwd_quant", "row_deq_inv", "col_inv"]
+    # one step = for each bit width the public two-sided forward call, then
+    # the inverse call; each call launches `npass` pass kernels, timed one by
+    # one with CUDA events the library records between its launches
+    npass = harp.harp_pass_count(left, right, cbs[0])
+    assert npass > 0, "the two-sided calls should run the pass kernels"
+    pass_fma = [harp.harp_pass_fma(left, right, cbs[0], k) for k in range(npass)]
+    names = [f"fwd_p{k}" for k in range(npass)] + [f"inv_p{k}" for k in range(npass)]
     kt = {f"{n}_{b}bit": [] for b in BITS for n in names}
+    ev_pool = []
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)                     # creates the CUDA event before timing
+        return evs
 
     def step(record):
         evs = []
         for cb, (codes, scales) in zip(cbs, outs):
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
             if record:
-                e[0].record(stream)
-            harp.harp_rotate(left, harp.HARP_LEFT, harp.HARP_FWD, x, ws, stream)
+                ef, ei = ev_pool.pop(), ev_pool.pop()
+                harp.harp_set_pass_events(ef)
+            harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws, stream)
             if record:
-                e[1].record(stream)
-            harp.harp_rotate_quantize(None, right, cb, ws, codes, scales, None, None, stream)
+                harp.harp_set_pass_events(ei)
+            harp.harp_dequantize_unrotate(left, right, cb, codes, scales, out, ws, stream)
             if record:
-                e[2].record(stream)
-            harp.harp_dequantize_unrotate(None, right, cb, codes, scales, ws, None, stream)
-            if record:
-                e[3].record(stream)
-            harp.harp_rotate(left, harp.HARP_LEFT, harp.HARP_INV, ws, out, stream)
-            if record:
-                e[4].record(stream)
-                evs.append((cb.bits, e))
+                harp.harp_set_pass_events([])
+                evs.append((cb.bits, ef, ei))
         return evs
+
+    for _ in range(2 * len(BITS) * args.steps):
+        ev_pool.append(new_events(npass + 1))
+    torch.cuda.synchronize()
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -212,9 +222,10 @@ def run_gpu(args, rank, world, local_rank):
     clk = clocks.stop()
     for s0, s1, evs in all_evs:
         step_ms.append(s0.elapsed_time(s1))
-        for bits, e in evs:
-            for i, n in enumerate(names):
-                kt[f"{n}_{bits}bit"].append(e[i].elapsed_time(e[i + 1]))
+        for bits, ef, ei in evs:
+            for k in range(npass):
+                kt[f"fwd_p{k}_{bits}bit"].append(ef[k].elapsed_time(ef[k + 1]))
+                kt[f"inv_p{k}_{bits}bit"].append(ei[k].elapsed_time(ei[k + 1]))
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -267,10 +278,16 @@ def run_gpu(args, rank, world, local_rank):
                "api": "harp_rotate_quantize + harp_dequantize_unrotate (two-sided), pinned host buffers",
                "workspace_bytes": ws_bytes}
     del flush
-    return total_ms, step_ms, kt, clk, e2e
+    return total_ms, step_ms, kt, clk, e2e, npass, pass_fma
 
 
-def kernel_table(kt):
+def kernel_table(kt, npass, pass_fma):
+    """Per pass kernel: mean duration, the bytes it moves itself (input read,
+    output written: bf16 weight, fp32 workspace, codes + scales), the
+    algorithmic bytes of the step it accounts for, and its FLOP rate: forward
+    pass k applies stages whose radices sum to pass_fma[k] (one FMA per block
+    coefficient per element, 2 flop each); inverse pass k applies the stages
+    of forward pass npass-1-k."""
     n = ROWS * COLS
     out = {}
     for key, v in kt.items():
@@ -279,19 +296,19 @@ def kernel_table(kt):
         us = 1e3 * statistics.mean(v)
         name, bits = key.rsplit("_", 1)
         b = int(bits[:-3])
-        if name == "col_fwd":
-            alg = n * 2.0                      # bf16 weight in (fp32 intermediate not credited)
-            own = n * (2.0 + 4.0)
-        elif name == "row_fwd_quant":
-            alg = n * (b / 8.0 + 2.0 / GROUP)  # codes + scales out
-            own = n * (4.0 + b / 8.0 + 2.0 / GROUP)
-        elif name == "row_deq_inv":
-            alg = n * (b / 8.0 + 2.0 / GROUP)
-            own = n * (b / 8.0 + 2.0 / GROUP + 4.0)
+        kind, pk = name.split("_p")
+        k = int(pk)
+        flop = n * 2 * (pass_fma[k] if kind == "fwd" else pass_fma[npass - 1 - k])
+        code_b = b / 8.0 + 2.0 / GROUP
+        if kind == "fwd":
+            rd = 2.0 if k == 0 else 4.0
+            wr = code_b if k == npass - 1 else 4.0
+            alg = n * (2.0 if k == 0 else 0.0) + n * (code_b if k == npass - 1 else 0.0)
         else:
-            alg = n * 2.0
-            own = n * (4.0 + 2.0)
-        flop = n * FLOP_PER_ELEM_SIDE
+            rd = code_b if k == 0 else 4.0
+            wr = 2.0 if k == npass - 1 else 4.0
+            alg = n * (code_b if k == 0 else 0.0) + n * (2.0 if k == npass - 1 else 0.0)
+        own = n * (rd + wr)
         out[key] = {"us": round(us, 2), "own_bytes": int(own), "own_gbs": round(own / (us * 1e-6) / 1e9, 1),
                     "alg_bytes": int(alg), "tflops": round(flop / (us * 1e-6) / 1e12, 2)}
     return out
@@ -401,13 +418,13 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    total_ms, step_ms, kt, clk, e2e = run_gpu(args, rank, world, local_rank)
+    total_ms, step_ms, kt, clk, e2e, npass, pass_fma = run_gpu(args, rank, world, local_rank)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         value = world * STEP_BYTES * args.steps / (total_ms * 1e-3) / 1e9
-        ktab = kernel_table(kt)
+        ktab = kernel_table(kt, npass, pass_fma)
         # dominant kernel: largest total time in the step
         dom = max(ktab, key=lambda k: ktab[k]["us"])
         smhz = float(peaks.get("sm_max_mhz", 1965.0))
@@ -416,7 +433,7 @@ def main():
         roof = {"kernel": dom, "bound": "alu", "achieved": d["tflops"], "peak": round(peak_tf, 1),
                 "unit": "TFLOP/s", "frac": round(d["tflops"] / peak_tf, 4), "traffic": None,
                 "peak_source": f"FFMA: 148 SM x 128 lanes x 2 flop x {smhz:.0f} MHz (max SM clock, {peak_src})",
-                "algorithmic": f"{FLOP_PER_ELEM_SIDE} flop per element per side ({sum(RADIX)} FMA)",
+                "algorithmic": f"2 flop per block coefficient per element: FMA per element by forward pass {pass_fma}",
                 "own_bytes_hbm_frac": round(d["own_gbs"] / hbm, 4)}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -435,7 +452,7 @@ def main():
                            "step_bytes": int(STEP_BYTES)},
                 "hbm_frac": round(value / world / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": peak_src,
                 "roofline": roof, "kernels": ktab, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 8 * args.steps, "clocks": clk}
+                "gpu_launches": 2 * len(BITS) * npass * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -172,8 +172,9 @@ int harp_codebook_destroy(harp_codebook_t cb);
 int harp_codebook_tables(harp_codebook_t cb, float *centroids, float *thresholds);
 
 /* Bytes of device workspace the fused two-sided calls need for a
- * [rows x cols] matrix: rows*cols*4 (an fp32 intermediate) when `left` is
- * not NULL, else 0. */
+ * [rows x cols] matrix: rows*cols*8 (two fp32 intermediates, between which
+ * the passes of the two-sided path alternate) when `left` is not NULL,
+ * else 0. */
 int harp_workspace_size(harp_plan_t left, harp_plan_t right, int64_t rows, int64_t cols,
                         size_t *bytes);
 
@@ -229,11 +230,33 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
                              int64_t cols, void *out, int out_dtype, void *workspace,
                              size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------------------ timing hooks */
+
+/* Number of kernel launches (passes) harp_rotate_quantize and
+ * harp_dequantize_unrotate make for this pair of processors and codebook
+ * when both sides are given; 0 when they fall back to one launch per side.
+ * Host-only. */
+int harp_pass_count(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int *passes);
+
+/* FMAs per matrix element that pass `pass` (0-based, forward order) of the
+ * two-sided plan spends: the sum of the radices of the stages it applies
+ * (pass np-1-k of the inverse call applies the same stages). Host-only.
+ * Errors: INVALID_ARG (NULL argument, no pass plan, pass out of range). */
+int harp_pass_fma(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int pass, int *fma);
+
+/* Register CUDA events (cudaEvent_t handles, owned by the caller and kept
+ * alive while registered) for timing the passes of the fused two-sided
+ * calls made afterwards by the calling thread: each such call records
+ * events[0] on its stream before its first pass and events[k+1] after pass k
+ * (for k + 1 < n). n = 0 unregisters. No effect on results. Errors:
+ * INVALID_ARG (n < 0, or NULL events with n > 0). */
+int harp_set_pass_events(void *const *events, int n);
+
 /* ------------------------------------------- variant that allocates nothing */
 
 /* Capacity of the library-owned scratch used by harp_rotate_quantize_static:
- * 32 MiB, i.e. a two-sided matrix of up to 8,388,608 elements (for example
- * 2048 x 4096). */
+ * 32 MiB, i.e. a two-sided matrix of up to 4,194,304 elements (for example
+ * 2048 x 2048 or 1024 x 4096; harp_workspace_size gives the need). */
 #define HARP_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
 
 /* harp_rotate_quantize without a caller workspace. The pages have no
@@ -249,7 +272,7 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
  * inside the library, which every device that loads the library holds until
  * the process exits. The call allocates no memory (no cudaMalloc / cudaFree,
  * no allocating library routine).
- *  - Size limit: rows*cols*4 bytes (harp_workspace_size) above
+ *  - Size limit: a workspace need (harp_workspace_size, rows*cols*8 bytes) above
  *    HARP_STATIC_WORKSPACE_BYTES returns HARP_ERR_WORKSPACE before anything
  *    is launched. Right-only calls (left = NULL) need no scratch.
  *  - Set-up: the first two-sided call on a device looks up the array's

@@ -39,6 +39,7 @@ EXPORTS = (
     "harp_codebook_create", "harp_codebook_destroy", "harp_codebook_tables",
     "harp_workspace_size", "harp_rotate", "harp_quantize", "harp_dequantize",
     "harp_rotate_quantize", "harp_dequantize_unrotate", "harp_rotate_quantize_static",
+    "harp_pass_count", "harp_pass_fma", "harp_set_pass_events",
 )
 
 
@@ -82,6 +83,9 @@ def lib():
                                            ctypes.c_size_t, _P]
         L.harp_dequantize_unrotate.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _P, _INT, _P,
                                                ctypes.c_size_t, _P]
+        L.harp_pass_count.argtypes = [_P, _P, _P, ctypes.POINTER(_INT)]
+        L.harp_pass_fma.argtypes = [_P, _P, _P, _INT, ctypes.POINTER(_INT)]
+        L.harp_set_pass_events.argtypes = [_P, _INT]
         L.harp_rotate_quantize_static.argtypes = [_P, _P, _P, _P, _INT, _I64, _I64, _P, _P, _P, _P]
         _lib = L
     return _lib
@@ -266,6 +270,36 @@ def harp_rotate_quantize(left, right, cb, x, codes, scales, rotated_out=None, wo
                                       _ptr(rotated_out), _ptr(workspace), ws, _stream(stream)),
            "harp_rotate_quantize")
     return codes, scales
+
+
+def harp_pass_count(left, right, cb) -> int:
+    n = ctypes.c_int()
+    _check(lib().harp_pass_count(left.handle if left else None, right.handle, cb.handle, ctypes.byref(n)),
+           "harp_pass_count")
+    return n.value
+
+
+def harp_pass_fma(left, right, cb, k) -> int:
+    n = ctypes.c_int()
+    _check(lib().harp_pass_fma(left.handle, right.handle, cb.handle, k, ctypes.byref(n)), "harp_pass_fma")
+    return n.value
+
+
+_event_array = None
+
+
+def harp_set_pass_events(events):
+    """Time the passes of the following two-sided calls of this thread with
+    torch.cuda.Event objects (enable_timing=True); [] unregisters."""
+    global _event_array
+    handles = []
+    for e in events:
+        if e.cuda_event == 0:          # torch creates the CUDA event on first record
+            e.record()
+        handles.append(e.cuda_event)
+    _event_array = (ctypes.c_void_p * max(len(handles), 1))(*handles)
+    _check(lib().harp_set_pass_events(_event_array if handles else None, len(handles)),
+           "harp_set_pass_events")
 
 
 def harp_rotate_quantize_static(left, right, cb, x, codes, scales, rotated_out=None, stream=None):

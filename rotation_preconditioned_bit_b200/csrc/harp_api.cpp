@@ -413,7 +413,7 @@ int harp_workspace_size(harp_plan_t left, harp_plan_t right, int64_t rows, int64
                         size_t *bytes) {
     (void)right;
     if (!bytes || rows < 0 || cols < 0) return HARP_ERR_INVALID_ARG;
-    *bytes = left ? static_cast<size_t>(rows) * static_cast<size_t>(cols) * 4 : 0;
+    *bytes = left ? static_cast<size_t>(rows) * static_cast<size_t>(cols) * 8 : 0;
     return HARP_OK;
 }
 
@@ -493,7 +493,7 @@ static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, i
         harp::vec_tile(right->dev, harp::EPI_QUANT, cb->q.group) == 0)
         return HARP_ERR_UNSUPPORTED;
     if (left) {
-        const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(cols) * 4;
+        const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(cols) * 8;
         if (need && (!workspace || ws_bytes < need)) return HARP_ERR_WORKSPACE;
         if (workspace && !aligned(workspace, 16)) return HARP_ERR_ALIGNMENT;
     }
@@ -547,6 +547,26 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
     Lr.codes = codes;
     Lr.scales = scales;
     return cuda_status(harp::launch_vec(right->dev, &cb->q, Lr, stream));
+}
+
+int harp_pass_count(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int *passes) {
+    if (!right || !cb || !passes) return HARP_ERR_INVALID_ARG;
+    *passes = (left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group)) ? harp::pass_count(left->dev, right->dev, cb->q.group) : 0;
+    return HARP_OK;
+}
+
+int harp_pass_fma(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int pass, int *fma) {
+    if (!left || !right || !cb || !fma) return HARP_ERR_INVALID_ARG;
+    const int f = harp::pass_fma(left->dev, right->dev, cb->q.group, pass);
+    if (f < 0) return HARP_ERR_INVALID_ARG;
+    *fma = f;
+    return HARP_OK;
+}
+
+int harp_set_pass_events(void *const *events, int n) {
+    if (n < 0 || (n > 0 && !events)) return HARP_ERR_INVALID_ARG;
+    harp::set_pass_events(events, n);
+    return HARP_OK;
 }
 
 int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,

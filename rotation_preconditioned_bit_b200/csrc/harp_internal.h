@@ -83,12 +83,20 @@ int launch_dequantize(const QuantDev &q, const uint8_t *codes, const uint16_t *s
 // rows x cols workspace; every pass updates its tiles in place.
 // pass_plan_ok: whether such a plan exists for these processors and group.
 bool pass_plan_ok(const PlanDev &left, const PlanDev &right, int group);
+int pass_count(const PlanDev &left, const PlanDev &right, int group);
+// FMAs per element of forward pass k (sum of its radices), -1 if none.
+int pass_fma(const PlanDev &left, const PlanDev &right, int group, int k);
 int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q, const void *in,
                     int in_dtype, uint8_t *codes, uint16_t *scales, float *rotated_out, float *ws,
                     void *stream);
 int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q,
                     const uint8_t *codes, const uint16_t *scales, void *out, int out_dtype,
                     float *ws, void *stream);
+
+// Timing hook of the pass launchers (harp_set_pass_events): when n > 0,
+// every fused call records events[0] before its first pass and events[k+1]
+// after pass k (k + 1 < n). Per calling thread.
+void set_pass_events(void *const *events, int n);
 
 // Vectors per CTA the whole-vector kernel uses for this plan and epilogue
 // (0 if a vector does not fit in shared memory).

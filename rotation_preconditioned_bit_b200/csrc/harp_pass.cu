@@ -43,12 +43,36 @@ namespace {
 
 using namespace dq;
 
-constexpr int PT = 256;               // threads per CTA
+constexpr int PT = 512;               // threads per CTA (one CTA per SM)
 constexpr int PW = PT / 32;           // warps per CTA
 constexpr int MAXPS = 12;             // stages (both sides) in one pass
 constexpr int TILE_MAX = 16384;       // tile elements
-constexpr int SMEM_BUDGET = 112 * 1024;  // bytes per CTA: two CTAs per SM
+constexpr int SMEM_BUDGET = 232448;    // bytes per CTA (opt-in maximum): two tile buffers
 constexpr int GPAD = 4;               // floats between coefficient slots
+
+// Division by a fixed divisor d >= 1 as a multiply-high and a shift (exact
+// for dividends below 2^31): sh = ceil(log2 d), mul = 2^32 (2^sh - d) / d + 1.
+struct FDiv {
+    unsigned d, mul;
+    int sh;
+};
+
+inline FDiv make_fdiv(unsigned d) {
+    FDiv f;
+    f.d = d;
+    f.sh = 0;
+    while ((1u << f.sh) < d) ++f.sh;
+    f.mul = static_cast<unsigned>(((uint64_t(1) << 32) * ((uint64_t(1) << f.sh) - d)) / d + 1);
+    return f;
+}
+
+__host__ __device__ __forceinline__ unsigned fdiv(unsigned u, const FDiv &f) {
+#ifdef __CUDA_ARCH__
+    return (__umulhi(u, f.mul) + u) >> f.sh;
+#else
+    return static_cast<unsigned>((((static_cast<uint64_t>(u) * f.mul) >> 32) + u) >> f.sh);
+#endif
+}
 
 // One axis of a tile box. Global index of tile-local index i (tile position
 // hb, lb): (hb*Hx + hh)*P*S + mid*S + lb*Lx + ll with hh = i / (P*Lx),
@@ -62,6 +86,7 @@ struct PAxis {
     int64_t nlo;      // S / Lx
     int64_t nt;       // tile positions along the axis
     const float *sign;  // sign vector applied on this axis (nullptr: none)
+    FDiv f_nlo, f_PS, f_S, f_Hx, f_Lx;   // divisions by nlo, P*S, S, Hx, Lx
 };
 
 struct PStage {
@@ -81,12 +106,19 @@ struct PassDesc {
     int nst;
     PStage st[MAXPS];
     int TCp;            // tile pitch in floats (odd)
+    int buf_floats;     // floats per coefficient+table buffer (two buffers follow the tile)
+    int tile_floats;    // floats of the tile (first in shared memory)
+    int lev_base;       // float offset of the 16 dequantised levels
+    int loc_base;       // float offset of the per-pass local index tables (rows, then columns)
+    FDiv f_nch;         // division by the number of 32-column chunks of a tile row
     int coef_base;      // float offset of the coefficient area
     int coef_floats;
     int tab_base;       // float offset of the index tables (rows, then cols)
-    int stage_base;     // float offset of the code staging area (codes prologue)
     int smem_bytes;
     int sign_at_store;  // inverse: signs after the stages
+    int in_blocked;     // input is a workspace in this pass's tile-major layout
+    int out_blocked;    // output is a workspace in the next pass's tile-major layout
+    PAxis nx[2];        // the next pass's tile geometry (out_blocked)
     const void *in;
     int64_t ld_in;
     const uint8_t *in_codes;
@@ -99,50 +131,89 @@ struct PassDesc {
     int64_t cols;       // matrix columns (row strides of codes, scales, copy)
 };
 
-__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem));
-}
-
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
 }
 
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Global index along axis A of tile-local index i at tile position pos
+// (32-bit: every index is below the axis length d < 2^31).
+__host__ __device__ __forceinline__ int axis_global(const PAxis &A, unsigned pos, int i) {
+    const unsigned nlo = static_cast<unsigned>(A.nlo), S = static_cast<unsigned>(A.S);
+    const unsigned hb = pos / nlo, lb = pos - hb * nlo;
+    const unsigned pl = static_cast<unsigned>(A.P * A.Lx);
+    const unsigned hh = static_cast<unsigned>(i) / pl, rem = static_cast<unsigned>(i) - hh * pl;
+    const unsigned mid = rem / A.Lx, ll = rem - mid * A.Lx;
+    return static_cast<int>((hb * A.Hx + hh) * A.P * S + mid * S + lb * A.Lx + ll);
 }
 
-__host__ __device__ __forceinline__ int axis_global(const PAxis &A, int64_t pos, int i) {
-    const int64_t hb = pos / A.nlo, lb = pos - hb * A.nlo;
-    const int pl = A.P * A.Lx;
-    const int hh = i / pl, rem = i - hh * pl;
-    const int mid = rem / A.Lx, ll = rem - mid * A.Lx;
-    return static_cast<int>((hb * A.Hx + hh) * A.P * A.S + mid * A.S + lb * A.Lx + ll);
+// Inverse of axis_global: tile position and tile-local index of global
+// index i.
+__host__ __device__ __forceinline__ void axis_local(const PAxis &A, int i, unsigned &pos, int &loc) {
+    const unsigned u = static_cast<unsigned>(i);
+    const unsigned hi = fdiv(u, A.f_PS), rem = u - hi * A.f_PS.d;
+    const unsigned mid = fdiv(rem, A.f_S), lo = rem - mid * A.f_S.d;
+    const unsigned hb = fdiv(hi, A.f_Hx), hh = hi - hb * A.Hx, lb = fdiv(lo, A.f_Lx), ll = lo - lb * A.Lx;
+    pos = hb * static_cast<unsigned>(A.nlo) + lb;
+    loc = static_cast<int>((hh * A.P + mid) * A.Lx + ll);
+}
+
+// Global index of the first element (local index 0) of the tile at
+// position pos; local index i adds axis_global(A, 0, i) - axis_global(A, 0, 0).
+__host__ __device__ __forceinline__ int axis_base(const PAxis &A, unsigned pos) {
+    const unsigned hb = fdiv(pos, A.f_nlo), lb = pos - hb * static_cast<unsigned>(A.nlo);
+    return static_cast<int>(hb * A.Hx * A.f_PS.d + lb * A.Lx);
 }
 
 // Global group index (c = h*s + l) of tile group gi of stage S.
-__host__ __device__ __forceinline__ int64_t global_group(const PStage &S, const int *tab, int gi) {
+__host__ __device__ __forceinline__ int global_group(const PStage &S, const int *tab, int gi) {
     const int base = (gi / S.sig) * (S.b * S.sig) + gi % S.sig;
-    const int64_t i = tab[base];
-    const int64_t bs = static_cast<int64_t>(S.b) * S.s;
-    const int64_t h = i / bs;
-    return h * S.s + (i - h * bs) % S.s;
+    const unsigned i = static_cast<unsigned>(tab[base]);
+    const unsigned s = static_cast<unsigned>(S.s), bs = static_cast<unsigned>(S.b) * s;
+    const unsigned h = i / bs;
+    return static_cast<int>(h * s + (i - h * bs) % s);
 }
 
 // ------------------------------------------------------------ one stage
 
-// Tile addresses of one lane's 4 vectors of group gi (inputs j = 0 at p[v]),
-// and its coefficient slot. Lanes past the last group or vector are clamped
-// onto valid data and store nothing.
+// Packed fp32 pairs (two IEEE single-precision FMAs per instruction; each
+// half rounds exactly like fmaf).
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t f2_pack(float lo, float hi) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(f2_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Vectors per lane in a stage work unit.
+constexpr int VL = 2;
+
+// Tile addresses of one lane's VL vectors of group gi (inputs j = 0 at
+// p[v]), and its coefficient slot. Lanes past the last group or vector are
+// clamped onto valid data and store nothing.
 __device__ __forceinline__ void unit_addr(const PStage &S, int gi, int v0, int LV, int NV, int A, int Bv,
-                                          const float *Cs, int (&p)[4], bool (&vok)[4], bool &gok,
+                                          const float *Cs, int (&p)[VL], bool (&vok)[VL], bool &gok,
                                           const float *&wp) {
     gok = gi < S.G;
     const int g = gok ? gi : S.G - 1;
     const int base = (g / S.sig) * (S.b * S.sig) + g % S.sig;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < VL; ++v) {
         const int vi = v0 + LV * v;
         vok[v] = vi < NV;
         p[v] = base * A + min(vi, NV - 1) * Bv;
@@ -150,33 +221,38 @@ __device__ __forceinline__ void unit_addr(const PStage &S, int gi, int v0, int L
     wp = Cs + g * S.gstride;
 }
 
-// acc[k][v] = sum_j w[j][k] * x_v[j] for K outputs and 4 vectors. Inputs
-// past b are read at b-1 and meet zero coefficients.
-template <int K>
+// acc[q][v] = (out 2q, out 2q+1) of vector v: sum_j w[j][k] * x_v[j] for K
+// outputs and VL vectors, as packed pairs of outputs (the coefficient row
+// w[j][0..K) is read as K/4 16-byte words = K/2 pairs; x_v[j] is broadcast
+// into both halves). CLAMP: inputs past b are read at b-1 and meet zero
+// coefficients (only when b is not a multiple of 4).
+template <int K, bool CLAMP>
 __device__ __forceinline__ void unit_compute(const float *T, const float *wp, int kp, int jpad, int b,
-                                             int step, const int (&p)[4], float (&acc)[K][4]) {
+                                             int step, const int (&p)[VL], f2_t (&acc)[K / 2][VL]) {
 #pragma unroll
-    for (int k = 0; k < K; ++k)
+    for (int q = 0; q < K / 2; ++q)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) acc[k][v] = 0.0f;
+        for (int v = 0; v < VL; ++v) acc[q][v] = 0ull;
     for (int j0 = 0; j0 < jpad; j0 += 4) {
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const int j = j0 + jj;
-            const int off = min(j, b - 1) * step;
-            float x[4];
+            const int off = (CLAMP ? min(j, b - 1) : j) * step;
+            f2_t x[VL];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) x[v] = T[p[v] + off];
+            for (int v = 0; v < VL; ++v) {
+                const float xv = T[p[v] + off];
+                x[v] = f2_pack(xv, xv);
+            }
             const float4 *w4 = reinterpret_cast<const float4 *>(wp + j * kp);
 #pragma unroll
             for (int q = 0; q < K / 4; ++q) {
                 const float4 w = w4[q];
+                const f2_t wa = f2_pack(w.x, w.y), wb = f2_pack(w.z, w.w);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    acc[4 * q + 0][v] = fmaf(w.x, x[v], acc[4 * q + 0][v]);
-                    acc[4 * q + 1][v] = fmaf(w.y, x[v], acc[4 * q + 1][v]);
-                    acc[4 * q + 2][v] = fmaf(w.z, x[v], acc[4 * q + 2][v]);
-                    acc[4 * q + 3][v] = fmaf(w.w, x[v], acc[4 * q + 3][v]);
+                for (int v = 0; v < VL; ++v) {
+                    acc[2 * q][v] = f2_fma(wa, x[v], acc[2 * q][v]);
+                    acc[2 * q + 1][v] = f2_fma(wb, x[v], acc[2 * q + 1][v]);
                 }
             }
         }
@@ -184,22 +260,26 @@ __device__ __forceinline__ void unit_compute(const float *T, const float *wp, in
 }
 
 template <int K>
-__device__ __forceinline__ void unit_store(float *T, int b, int k0, int step, const int (&p)[4],
-                                           const bool (&vok)[4], bool gok, const float (&acc)[K][4]) {
+__device__ __forceinline__ void unit_store(float *T, int b, int k0, int step, const int (&p)[VL],
+                                           const bool (&vok)[VL], bool gok, const f2_t (&acc)[K / 2][VL]) {
     if (!gok) return;
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-        if (k0 + k < b) {
+    for (int v = 0; v < VL; ++v) {
+        if (!vok[v]) continue;
+        float *y = T + p[v] + k0 * step;
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-                if (vok[v]) T[p[v] + (k0 + k) * step] = acc[k][v];
+        for (int q = 0; q < K / 2; ++q) {
+            float lo, hi;
+            f2_unpack(acc[q][v], lo, hi);
+            if (k0 + 2 * q < b) y[(2 * q) * step] = lo;
+            if (k0 + 2 * q + 1 < b) y[(2 * q + 1) * step] = hi;
         }
     }
 }
 
 // One stage over the whole tile. A / Bv: tile address steps along the
 // group axis / the vector axis; NV: vectors. Work units are (block of 32/LV
-// groups, 4*LV vectors); with b <= 16 (one chunk of K outputs) every unit
+// groups, VL*LV vectors); with b <= 16 (one chunk of K outputs) every unit
 // reads and writes only its own elements, so units update the tile in place
 // without barriers. Wider blocks (ROUNDS) split the outputs into chunks of K
 // over several warps, which first all read (compute into registers), then
@@ -209,22 +289,24 @@ __device__ __forceinline__ void stage_run(float *T, const float *C, const PStage
                                           int warp, int lane) {
     const int LV = S.LV, LG = 32 / LV;
     const int lv = lane & (LV - 1), lg = lane / LV;
-    const int span = LV * 4;
+    const int span = LV * VL;
     const int nvc = (NV + span - 1) / span;
     const int ngb = (S.G + LG - 1) / LG;
     const int nkc = S.kp / K;
     const int step = S.sig * A;
+    const bool clamp = (S.jpad != S.b);
     const float *Cs = C + S.coff;
     if constexpr (!ROUNDS) {
         const int nunits = ngb * nvc;
         for (int u = warp; u < nunits; u += PW) {
             const int gb = u / nvc, vc = u - gb * nvc;
-            int p[4];
-            bool vok[4], gok;
+            int p[VL];
+            bool vok[VL], gok;
             const float *wp;
             unit_addr(S, gb * LG + lg, vc * span + lv, LV, NV, A, Bv, Cs, p, vok, gok, wp);
-            float acc[K][4];
-            unit_compute<K>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
+            f2_t acc[K / 2][VL];
+            if (clamp) unit_compute<K, true>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
+            else unit_compute<K, false>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
             unit_store<K>(T, S.b, 0, step, p, vok, gok, acc);
         }
     } else {
@@ -234,14 +316,16 @@ __device__ __forceinline__ void stage_run(float *T, const float *C, const PStage
         for (int r = 0; r < nrounds; ++r) {
             const int blk = r * bpr + warp / nkc, kc = warp - (warp / nkc) * nkc;
             const bool active = (warp < bpr * nkc) && (blk < nblk);
-            float acc[K][4];
-            int p[4] = {0, 0, 0, 0};
-            bool vok[4] = {false, false, false, false}, gok = false;
+            f2_t acc[K / 2][VL];
+            int p[VL];
+            bool vok[VL], gok = false;
+#pragma unroll
+            for (int v = 0; v < VL; ++v) { p[v] = 0; vok[v] = false; }
             if (active) {
                 const int gb = blk / nvc, vc = blk - gb * nvc;
                 const float *wp;
                 unit_addr(S, gb * LG + lg, vc * span + lv, LV, NV, A, Bv, Cs, p, vok, gok, wp);
-                unit_compute<K>(T, wp + kc * K, S.kp, S.jpad, S.b, step, p, acc);
+                unit_compute<K, true>(T, wp + kc * K, S.kp, S.jpad, S.b, step, p, acc);
             }
             __syncthreads();
             if (active) unit_store<K>(T, S.b, kc * K, step, p, vok, gok, acc);
@@ -250,43 +334,30 @@ __device__ __forceinline__ void stage_run(float *T, const float *C, const PStage
     }
 }
 
+// Stages with blocks wider than 16 (rare) run out of line so that their
+// barrier-separated rounds do not raise the register pressure of the rest.
+__device__ __noinline__ void stage_rounds(float *T, const float *C, const PStage &S, int A, int Bv, int NV,
+                                          int warp, int lane) {
+    stage_run<8, true>(T, C, S, A, Bv, NV, warp, lane);
+}
+
 // ------------------------------------------------------------ prologue / epilogue
 
-constexpr int MAXQ = 16;   // bf16 pairs per lane when a tile row is expanded (Ec <= 1024)
 
-// Forward-side sign factors of tile row tr / column tc (1 when none).
-__device__ __forceinline__ float row_sign(const PassDesc &D, const int *rtab, int tr) {
-    return D.ax[0].sign ? __ldg(D.ax[0].sign + rtab[tr]) : 1.0f;
-}
-__device__ __forceinline__ float col_sign(const PassDesc &D, const int *ctab, int tc) {
-    return D.ax[1].sign ? __ldg(D.ax[1].sign + ctab[tc]) : 1.0f;
-}
-
-// Codes -> values for the first inverse pass: the packed words of the tile
-// (staged in shared memory) and its scales; 32 codes of one row per warp step.
-template <int BITS>
-__device__ __forceinline__ void decode_tile(float *T, const PassDesc &D, const QuantDev &Q, const uint32_t *cw,
-                                            const float *ssc, const float *lev, int warp, int lane) {
-    constexpr unsigned MASK = (1u << BITS) - 1u;
-    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
-    const int nch = Ec >> 5, wpr = nch * BITS, ngt = Ec / Q.group;
-    const int bit = lane * BITS, wi = bit >> 5, sh = bit & 31;
-    for (int u = warp; u < Er * nch; u += PW) {
-        const int tr = u / nch, ch = u - tr * nch;
-        const unsigned w = (lane < BITS) ? cw[tr * wpr + ch * BITS + lane] : 0u;
-        const unsigned w0 = __shfl_sync(FULL, w, wi);
-        const unsigned w1 = __shfl_sync(FULL, w, min(wi + 1, BITS - 1));
-        unsigned code = w0 >> sh;
-        if (sh + BITS > 32) code |= w1 << (32 - sh);
-        const float s = ssc[tr * ngt + (ch * 32) / Q.group];
-        T[tr * TCp + ch * 32 + lane] = s * lev[code & MASK];
-    }
-}
+// Per-tile index tables in shared memory (built once per tile): global row
+// offset (row * ld) and global column of every tile row / column, and the
+// sign factor of each when the pass applies the sign vectors.
+struct Tabs {
+    const int64_t *rin, *rout;    // per tile row: input / output offset of its first element
+    const int *rtab, *ctab;       // global row / column of each tile row / column
+    const int *cin, *cout;        // per tile column: input / output offset
+    const float *rsg, *csg;
+};
 
 // Scale, code and pack every (row, group) of the tile (last forward pass).
 template <int BITS, bool F32COPY>
 __device__ __forceinline__ void quantize_tile(const float *T, const PassDesc &D, const QuantDev &Q,
-                                              const int *rtab, const int *ctab, int warp, int lane) {
+                                              const Tabs &tb, int warp, int lane) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     const int g = Q.group, ngt = Ec / g, per = g >> 5;
     const bool is_max = (Q.kind == HARP_ABSMAX);
@@ -295,6 +366,7 @@ __device__ __forceinline__ void quantize_tile(const float *T, const PassDesc &D,
     for (int k = 0; k < (1 << BITS) - 1; ++k) t[k] = Q.thr[k];
     const int64_t spr = D.cols / g;
     const int64_t wpr = D.cols * BITS / 32;
+    const int c0t = tb.ctab[0];
     uint32_t *cw = reinterpret_cast<uint32_t *>(D.codes);
     for (int u = warp; u < Er * ngt; u += PW) {
         const int tr = u / ngt, gq = u - tr * ngt;
@@ -305,163 +377,471 @@ __device__ __forceinline__ void quantize_tile(const float *T, const PassDesc &D,
         const unsigned short hb = group_scale_bits(tot, Q);
         const float s = __half2float(__ushort_as_half(hb));
         const float inv = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
-        const int64_t row = rtab[tr];
-        const int64_t c0 = ctab[0] + gq * g;
+        const int64_t row = tb.rtab[tr];
+        const int64_t c0 = c0t + gq * g;
         if (lane == 0) D.scales[row * spr + c0 / g] = hb;
+        uint32_t *wrow = cw + row * wpr + (c0 / 32) * BITS;
+        float *frow = F32COPY ? D.out_f32 + row * D.cols + c0 : nullptr;
         for (int e = 0; e < per; ++e) {
             const float x = rp[lane + 32 * e];
             const int code = code_of<BITS>(x, s, inv, !is_max, t);
             const unsigned word = pack_words<BITS>(code, lane);
-            if (lane < BITS) cw[row * wpr + (c0 / 32 + e) * BITS + lane] = word;
-            if constexpr (F32COPY) D.out_f32[row * D.cols + c0 + 32 * e + lane] = x;
+            if (lane < BITS) wrow[e * BITS + lane] = word;
+            if constexpr (F32COPY) frow[32 * e + lane] = x;
+        }
+    }
+}
+
+// Tile <-> global moves in units of 4 rows x 32 columns per warp: lane
+// (q = lane / 8, c = lane % 8) moves 4 consecutive columns (16 contiguous
+// bytes of fp32, 8 of bf16: runs of tile columns are multiples of 4 and
+// aligned) of row 4u + q. With an odd pitch the 32 lanes of each shared
+// access hit 32 different banks.
+struct Quad {
+    int tr, tc;
+    bool ok;
+};
+
+__device__ __forceinline__ Quad quad_of(int u, const FDiv &fnch, int Er, int Ec, int lane) {
+    const int rq = static_cast<int>(fdiv(static_cast<unsigned>(u), fnch)), ch = u - rq * static_cast<int>(fnch.d);
+    Quad qd;
+    qd.tr = 4 * rq + (lane >> 3);
+    qd.tc = 32 * ch + 4 * (lane & 7);
+    qd.ok = qd.tr < Er && qd.tc < Ec;
+    return qd;
+}
+
+// Shared tile -> global (fp32 or bf16), times the sign factors when asked.
+// A quad goes out as one 16-byte (8-byte) store when its four outputs are
+// consecutive and aligned in the output layout, else element by element.
+template <int EPI>
+__device__ __forceinline__ void store_tile(const float *T, const PassDesc &D, const Tabs &tb, bool signs,
+                                           int warp, int lane) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
+    const int nch = (Ec + 31) >> 5, nu = ((Er + 3) >> 2) * nch;
+    for (int u = warp; u < nu; u += PW) {
+        const Quad qd = quad_of(u, D.f_nch, Er, Ec, lane);
+        if (!qd.ok) continue;
+        const float *t = T + qd.tr * TCp + qd.tc;
+        float4 x = make_float4(t[0], t[1], t[2], t[3]);
+        if (signs) {
+            const float rs = tb.rsg[qd.tr];
+            x.x *= rs * tb.csg[qd.tc];
+            x.y *= rs * tb.csg[qd.tc + 1];
+            x.z *= rs * tb.csg[qd.tc + 2];
+            x.w *= rs * tb.csg[qd.tc + 3];
+        }
+        const int c0 = tb.cout[qd.tc];
+        const int64_t off = tb.rout[qd.tr] + c0;
+        const bool vec = (tb.cout[qd.tc + 3] == c0 + 3) && ((off & 3) == 0);
+        if constexpr (EPI == EPI_BF16) {
+            unsigned short *o = static_cast<unsigned short *>(D.out);
+            const unsigned short b0 = __bfloat16_as_ushort(__float2bfloat16_rn(x.x));
+            const unsigned short b1 = __bfloat16_as_ushort(__float2bfloat16_rn(x.y));
+            const unsigned short b2 = __bfloat16_as_ushort(__float2bfloat16_rn(x.z));
+            const unsigned short b3 = __bfloat16_as_ushort(__float2bfloat16_rn(x.w));
+            if (vec) {
+                *reinterpret_cast<uint2 *>(o + off) =
+                    make_uint2(b0 | (static_cast<unsigned>(b1) << 16), b2 | (static_cast<unsigned>(b3) << 16));
+            } else {
+                const int64_t r = tb.rout[qd.tr];
+                o[r + c0] = b0;
+                o[r + tb.cout[qd.tc + 1]] = b1;
+                o[r + tb.cout[qd.tc + 2]] = b2;
+                o[r + tb.cout[qd.tc + 3]] = b3;
+            }
+        } else {
+            float *o = static_cast<float *>(D.out);
+            if (vec) {
+                *reinterpret_cast<float4 *>(o + off) = x;
+            } else {
+                const int64_t r = tb.rout[qd.tr];
+                o[r + c0] = x.x;
+                o[r + tb.cout[qd.tc + 1]] = x.y;
+                o[r + tb.cout[qd.tc + 2]] = x.z;
+                o[r + tb.cout[qd.tc + 3]] = x.w;
+            }
+        }
+    }
+}
+
+// Quantiser for 2- and 4-bit codes with groups of a multiple of 32: lane
+// (q = lane / 4, c = lane % 4) codes 8 consecutive values of row 8u + q, so
+// its 8 codes fill one 32-bit word (4 bits) or half of one (2 bits, joined
+// with the neighbouring lane's half). The group statistic adds each lane's
+// values in column order, then combines the lanes of the row with a fixed
+// xor tree.
+template <int BITS, bool F32COPY>
+__device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDesc &D, const QuantDev &Q,
+                                                   const Tabs &tb, int warp, int lane) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
+    const int g = Q.group, ngt = Ec / g, nit = g >> 5;
+    const bool is_max = (Q.kind == HARP_ABSMAX);
+    float t[(1 << BITS) - 1];
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) t[k] = Q.thr[k];
+    const int64_t spr = D.cols / g;
+    const int64_t wpr = D.cols * BITS / 32;
+    const int q = lane >> 2, c = lane & 3;
+    const int nro = (Er + 7) >> 3;
+    uint32_t *cw = reinterpret_cast<uint32_t *>(D.codes);
+    for (int u = warp; u < nro * ngt; u += PW) {
+        const int ro = u / ngt, gq = u - ro * ngt;
+        const int tr = 8 * ro + q;
+        const bool ok = tr < Er;
+        const float *rp = T + min(tr, Er - 1) * TCp + gq * g + 8 * c;
+        float st = 0.0f;
+        for (int it = 0; it < nit; ++it) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) st = combine(st, rp[32 * it + e], is_max);
+        }
+        float o = __shfl_xor_sync(FULL, st, 1);
+        st = is_max ? fmaxf(st, o) : st + o;
+        o = __shfl_xor_sync(FULL, st, 2);
+        st = is_max ? fmaxf(st, o) : st + o;
+        const unsigned short hb = group_scale_bits(st, Q);
+        const float s = __half2float(__ushort_as_half(hb));
+        const float inv = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+        const int64_t row = tb.rtab[min(tr, Er - 1)];
+        const int64_t c0 = tb.ctab[0] + gq * g;
+        if (ok && c == 0) D.scales[row * spr + c0 / g] = hb;
+        for (int it = 0; it < nit; ++it) {
+            unsigned word = 0;
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                x[e] = rp[32 * it + e];
+                word |= static_cast<unsigned>(code_of<BITS>(x[e], s, inv, !is_max, t)) << (BITS * e);
+            }
+            const int64_t col = c0 + 32 * it + 8 * c;       // first of this lane's 8 columns
+            if constexpr (BITS == 4) {
+                if (ok) cw[row * wpr + col / 8] = word;
+            } else {
+                const unsigned hi = __shfl_down_sync(FULL, word, 1);
+                if (ok && (c & 1) == 0) cw[row * wpr + col / 16] = word | (hi << 16);
+            }
+            if constexpr (F32COPY) {
+                if (ok) {
+                    float4 *f = reinterpret_cast<float4 *>(D.out_f32 + row * D.cols + col);
+                    f[0] = make_float4(x[0], x[1], x[2], x[3]);
+                    f[1] = make_float4(x[4], x[5], x[6], x[7]);
+                }
+            }
         }
     }
 }
 
 // ------------------------------------------------------------ the kernel
 
-template <int PRO, int EPI>
-__global__ void __launch_bounds__(PT, 2)
-pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev Q) {
-    extern __shared__ float4 sm4[];
-    float *sm = reinterpret_cast<float *>(sm4);
-    float *T = sm;
-    float *C = sm + D.coef_base;
-    int *rtab = reinterpret_cast<int *>(sm + D.tab_base);
-    int *ctab = rtab + D.ax[0].E;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
-    const int64_t pos_c = blockIdx.x % D.ax[1].nt;
-    const int64_t pos_r = blockIdx.x / D.ax[1].nt;
+// One of the two tile buffers in shared memory: tile, coefficient slots,
+// and the tile's index tables.
+struct Buf {
+    float *T, *C;
+    Tabs tb;
+    int64_t *rin, *rout;
+    int *rtab, *ctab, *cin, *cout;
+    float *rsg, *csg, *ssc;
+};
 
-    for (int i = tid; i < Er; i += PT) rtab[i] = axis_global(D.ax[0], pos_r, i);
-    for (int i = tid; i < Ec; i += PT) ctab[i] = axis_global(D.ax[1], pos_c, i);
-    __syncthreads();
+__device__ __forceinline__ Buf buf_of(float *sm, const PassDesc &D, int b) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E;
+    Buf B;
+    float *base = sm + D.tile_floats + b * D.buf_floats;
+    B.T = sm;
+    B.C = base;
+    B.rin = reinterpret_cast<int64_t *>(base + D.tab_base);
+    B.rout = B.rin + Er;
+    B.rtab = reinterpret_cast<int *>(B.rout + Er);
+    B.ctab = B.rtab + Er;
+    B.cin = B.ctab + Ec;
+    B.cout = B.cin + Ec;
+    B.rsg = reinterpret_cast<float *>(B.cout + Ec);
+    B.csg = B.rsg + Er;
+    B.ssc = B.csg + Ec;
+    B.tb = Tabs{B.rin, B.rout, B.rtab, B.ctab, B.cin, B.cout, B.rsg, B.csg};
+    return B;
+}
 
-    // block coefficients of every stage of the pass (one group per warp step)
+// Index tables of tile t: global rows / columns, input and output offsets
+// (natural row-major with leading dimension ld, or a workspace in tile-major
+// order: this pass's for the input, the next pass's for the output), signs.
+__device__ __forceinline__ void build_tables(const PassDesc &D, const Buf &B, const int *rloc, const int *cloc,
+                                             unsigned t, int64_t ld, int tid) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E;
+    const unsigned ntc = static_cast<unsigned>(D.ax[1].nt);
+    const unsigned pr = t / ntc, pc = t - pr * ntc;
+    const int rb = axis_base(D.ax[0], pr), cb = axis_base(D.ax[1], pc);
+    const int64_t E = static_cast<int64_t>(Er) * Ec;
+    const int nEc = D.nx[1].E;
+    const int64_t nE = static_cast<int64_t>(D.nx[0].E) * nEc;
+    const unsigned nntc = static_cast<unsigned>(D.nx[1].nt);
+    for (int i = tid; i < Er; i += PT) {
+        const int r = rb + rloc[i];
+        B.rtab[i] = r;
+        B.rin[i] = D.in_blocked ? static_cast<int64_t>(t) * E + static_cast<int64_t>(i) * Ec
+                                : static_cast<int64_t>(r) * ld;
+        if (D.out_blocked) {
+            unsigned p;
+            int l;
+            axis_local(D.nx[0], r, p, l);
+            B.rout[i] = static_cast<int64_t>(p) * nntc * nE + static_cast<int64_t>(l) * nEc;
+        } else {
+            B.rout[i] = static_cast<int64_t>(r) * ld;
+        }
+        B.rsg[i] = D.ax[0].sign ? __ldg(D.ax[0].sign + r) : 1.0f;
+    }
+    for (int i = tid; i < Ec; i += PT) {
+        const int c = cb + cloc[i];
+        B.ctab[i] = c;
+        B.cin[i] = D.in_blocked ? i : c;
+        if (D.out_blocked) {
+            unsigned p;
+            int l;
+            axis_local(D.nx[1], c, p, l);
+            B.cout[i] = static_cast<int>(p * nE + l);
+        } else {
+            B.cout[i] = c;
+        }
+        B.csg[i] = D.ax[1].sign ? __ldg(D.ax[1].sign + c) : 1.0f;
+    }
+}
+
+// Block coefficients of every stage of a tile into a coefficient buffer
+// (asynchronous 16-byte copies; the tile's tables must be built).
+__device__ __forceinline__ void issue_coefs(const PassDesc &D, const Tabs &tb, float *C, int warp, int lane) {
     for (int u = 0; u < D.nst; ++u) {
         const PStage &S = D.st[u];
         const int cpg = S.jpad * S.kp / 4;
-        const int *tab = S.axis == 0 ? rtab : ctab;
+        const int *tab = S.axis == 0 ? tb.rtab : tb.ctab;
         for (int gi = warp; gi < S.G; gi += PW) {
-            const int64_t c = global_group(S, tab, gi);
-            const float *src = S.coef + c * (S.jpad * S.kp);
+            const int c = global_group(S, tab, gi);
+            const float *src = S.coef + static_cast<int64_t>(c) * (S.jpad * S.kp);
             float *dst = C + S.coff + gi * S.gstride;
             for (int o = lane; o < cpg; o += 32) cp_async16(dst + 4 * o, src + 4 * o);
         }
     }
+}
 
-    // the tile
-    float *lev = sm + D.stage_base;                 // codes prologue: 16 levels,
-    float *ssc = lev + 16;                          // the tile's scales,
-    uint32_t *cw = reinterpret_cast<uint32_t *>(ssc + ((Er * (Ec / max(Q.group, 1)) + 3) & ~3));  // its words
-    if constexpr (PRO == PRO_F32) {
-        const float *in = static_cast<const float *>(D.in);
-        for (int tr = warp; tr < Er; tr += PW) {
-            const float *src = in + static_cast<int64_t>(rtab[tr]) * D.ld_in;
-            float *dst = T + tr * TCp;
-            for (int tc = lane; tc < Ec; tc += 32) cp_async4(dst + tc, src + ctab[tc]);
+constexpr int MAXCH = 8;   // 32-code chunks per tile row for the codes input (Ec <= 256)
+
+template <int BITS>
+__device__ __forceinline__ void decode_rows(const PassDesc &D, const QuantDev &Q, float *T, const float *ssc,
+                                            const float *lev, int warp, int lane) {
+    constexpr unsigned MASK = (1u << BITS) - 1u;
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
+    const int nch = Ec >> 5, wpr = nch * BITS, ngt = Ec / Q.group;
+    const int bit = lane * BITS, wi = bit >> 5, sh = bit & 31;
+    for (int tr = warp; tr < Er; tr += PW) {
+        float *row = T + tr * TCp;
+        const unsigned *wsrc = reinterpret_cast<const unsigned *>(row + (Ec - wpr));
+        float val[MAXCH];
+#pragma unroll
+        for (int ch = 0; ch < MAXCH; ++ch) {
+            val[ch] = 0.0f;
+            if (ch < nch) {
+                const unsigned w0 = wsrc[ch * BITS + wi];
+                const unsigned w1 = (sh + BITS > 32) ? wsrc[ch * BITS + wi + 1] : 0u;
+                unsigned code = w0 >> sh;
+                if (sh + BITS > 32) code |= w1 << (32 - sh);
+                val[ch] = ssc[tr * ngt + (ch * 32) / Q.group] * lev[code & MASK];
+            }
         }
-    } else if constexpr (PRO == PRO_BF16) {
-        // raw bf16 pairs into the upper half of each tile row, expanded below
-        const int half = Ec >> 1;
-        const unsigned short *in = static_cast<const unsigned short *>(D.in);
-        for (int tr = warp; tr < Er; tr += PW) {
-            const unsigned short *src = in + static_cast<int64_t>(rtab[tr]) * D.ld_in;
-            float *dst = T + tr * TCp + half;
-            for (int q = lane; q < half; q += 32) cp_async4(dst + q, src + ctab[2 * q]);
-        }
-    } else {
-        const int nch = Ec >> 5, wpr = nch * Q.bits, ngt = Ec / Q.group;
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < MAXCH; ++ch)
+            if (ch < nch) row[ch * 32 + lane] = val[ch];
+    }
+}
+
+// The next tile's input travels in registers while the current tile is
+// computed: per thread NQR quads of 4 values (16 bytes of fp32, 8 of bf16),
+// or for packed codes NWR words and one scale.
+constexpr int NQR = 8;    // quads per thread: 16K-element tiles / 512 threads / 4
+constexpr int NWR = 4;    // code words per thread: 16K codes * 4 bits / 32 / 512
+
+struct Pre {
+    uint4 q[NQR];
+    unsigned w[NWR];
+    float sc;
+};
+
+template <int PRO>
+__device__ __forceinline__ void load_pre(const PassDesc &D, const QuantDev &Q, const Tabs &tb, Pre &R, int tid,
+                                         int warp, int lane) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E;
+    if constexpr (PRO == PRO_CODES) {
+        const int wpr = (Ec >> 5) * Q.bits, ngt = Ec / Q.group;
         const int64_t rw = D.cols * Q.bits / 32;
         const uint32_t *words = reinterpret_cast<const uint32_t *>(D.in_codes);
-        for (int tr = warp; tr < Er; tr += PW) {
-            const uint32_t *src = words + static_cast<int64_t>(rtab[tr]) * rw + (ctab[0] >> 5) * Q.bits;
-            for (int w = lane; w < wpr; w += 32) cp_async4(cw + tr * wpr + w, src + w);
-        }
-        const int64_t spr = D.cols / Q.group;
-        for (int i = tid; i < Er * ngt; i += PT) {
-            const int tr = i / ngt, q = i - tr * ngt;
-            ssc[i] = __half2float(__ushort_as_half(
-                __ldg(D.in_scales + static_cast<int64_t>(rtab[tr]) * spr + ctab[0] / Q.group + q)));
-        }
-        if (tid < 16) lev[tid] = Q.level[tid];
-    }
-    cp_async_wait_all();
-    __syncthreads();
-
-    if constexpr (PRO == PRO_BF16) {
-        const int half = Ec >> 1;
-        for (int tr = warp; tr < Er; tr += PW) {
-            float *row = T + tr * TCp;
-            const float rs = D.sign_at_store ? 1.0f : row_sign(D, rtab, tr);
-            unsigned w[MAXQ];
+        const int c0 = tb.ctab[0];
 #pragma unroll
-            for (int k = 0; k < MAXQ; ++k) {
-                const int q = lane + 32 * k;
-                w[k] = (q < half) ? __float_as_uint(row[half + q]) : 0u;
+        for (int k = 0; k < NWR; ++k) {
+            const int i = tid + PT * k;
+            R.w[k] = 0u;
+            if (i < Er * wpr) {
+                const int tr = i / wpr, w = i - tr * wpr;
+                R.w[k] = __ldg(words + static_cast<int64_t>(tb.rtab[tr]) * rw + (c0 >> 5) * Q.bits + w);
             }
-            __syncwarp();
+        }
+        R.sc = 0.0f;
+        if (tid < Er * ngt) {
+            const int tr = tid / ngt, q = tid - tr * ngt;
+            R.sc = __half2float(__ushort_as_half(
+                __ldg(D.in_scales + static_cast<int64_t>(tb.rtab[tr]) * (D.cols / Q.group) + c0 / Q.group + q)));
+        }
+    } else {
+        const int nch = (Ec + 31) >> 5, nu = ((Er + 3) >> 2) * nch;
 #pragma unroll
-            for (int k = 0; k < MAXQ; ++k) {
-                const int q = lane + 32 * k;
-                if (q < half) {
-                    float c0 = rs, c1 = rs;
-                    if (!D.sign_at_store && D.ax[1].sign) {
-                        c0 *= col_sign(D, ctab, 2 * q);
-                        c1 *= col_sign(D, ctab, 2 * q + 1);
-                    }
-                    row[2 * q] = __uint_as_float(w[k] << 16) * c0;
-                    row[2 * q + 1] = __uint_as_float(w[k] & 0xffff0000u) * c1;
+        for (int k = 0; k < NQR; ++k) {
+            const int u = warp + PW * k;
+            const Quad qd = quad_of(u, D.f_nch, Er, Ec, lane);
+            R.q[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (u < nu && qd.ok) {
+                const int64_t off = tb.rin[qd.tr] + tb.cin[qd.tc];
+                if constexpr (PRO == PRO_F32) {
+                    R.q[k] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(D.in) + off));
+                } else {
+                    const uint2 t = __ldg(reinterpret_cast<const uint2 *>(
+                        static_cast<const unsigned short *>(D.in) + off));
+                    R.q[k].x = t.x;
+                    R.q[k].y = t.y;
                 }
             }
         }
-        __syncthreads();
-    } else if constexpr (PRO == PRO_F32) {
-        if (!D.sign_at_store && (D.ax[0].sign || D.ax[1].sign)) {
-            for (int tr = warp; tr < Er; tr += PW) {
-                const float rs = row_sign(D, rtab, tr);
-                for (int tc = lane; tc < Ec; tc += 32) T[tr * TCp + tc] *= rs * col_sign(D, ctab, tc);
+    }
+}
+
+// Registers -> fp32 tile (forward sign factors applied when asked). The
+// codes input goes through the tail of each tile row: words first, then
+// every warp decodes its rows in place.
+template <int PRO>
+__device__ __forceinline__ void store_pre(const PassDesc &D, const QuantDev &Q, const Tabs &tb, float *T,
+                                          float *ssc, const float *lev, const Pre &R, bool signs, int tid,
+                                          int warp, int lane) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
+    if constexpr (PRO == PRO_CODES) {
+        const int wpr = (Ec >> 5) * Q.bits, ngt = Ec / Q.group;
+#pragma unroll
+        for (int k = 0; k < NWR; ++k) {
+            const int i = tid + PT * k;
+            if (i < Er * wpr) {
+                const int tr = i / wpr, w = i - tr * wpr;
+                reinterpret_cast<unsigned *>(T + tr * TCp + (Ec - wpr))[w] = R.w[k];
             }
+        }
+        if (tid < Er * ngt) ssc[tid] = R.sc;
+        __syncthreads();
+        if (Q.bits == 2) decode_rows<2>(D, Q, T, ssc, lev, warp, lane);
+        else if (Q.bits == 3) decode_rows<3>(D, Q, T, ssc, lev, warp, lane);
+        else decode_rows<4>(D, Q, T, ssc, lev, warp, lane);
+    } else {
+        const int nch = (Ec + 31) >> 5, nu = ((Er + 3) >> 2) * nch;
+#pragma unroll
+        for (int k = 0; k < NQR; ++k) {
+            const int u = warp + PW * k;
+            const Quad qd = quad_of(u, D.f_nch, Er, Ec, lane);
+            if (u < nu && qd.ok) {
+                float4 x;
+                if constexpr (PRO == PRO_F32) {
+                    x = make_float4(__uint_as_float(R.q[k].x), __uint_as_float(R.q[k].y),
+                                    __uint_as_float(R.q[k].z), __uint_as_float(R.q[k].w));
+                } else {
+                    x = make_float4(__uint_as_float(R.q[k].x << 16), __uint_as_float(R.q[k].x & 0xffff0000u),
+                                    __uint_as_float(R.q[k].y << 16), __uint_as_float(R.q[k].y & 0xffff0000u));
+                }
+                if (signs) {
+                    const float rs = tb.rsg[qd.tr];
+                    x.x *= rs * tb.csg[qd.tc];
+                    x.y *= rs * tb.csg[qd.tc + 1];
+                    x.z *= rs * tb.csg[qd.tc + 2];
+                    x.w *= rs * tb.csg[qd.tc + 3];
+                }
+                float *t = T + qd.tr * TCp + qd.tc;
+                t[0] = x.x;
+                t[1] = x.y;
+                t[2] = x.z;
+                t[3] = x.w;
+            }
+        }
+    }
+}
+
+// Persistent: each CTA walks the tiles blockIdx.x, + gridDim.x, ... The
+// next tile's input is loaded into registers and its coefficients copied
+// (asynchronously) into the other coefficient buffer before the current
+// tile's stages run, so memory latency overlaps the arithmetic.
+template <int PRO, int EPI>
+__global__ void __launch_bounds__(PT, 1)
+pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev Q) {
+    extern __shared__ float4 sm4[];
+    float *sm = reinterpret_cast<float *>(sm4);
+    float *T = sm;
+    float *lev = sm + D.lev_base;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
+    const bool has_sign = D.ax[0].sign || D.ax[1].sign;
+    const bool load_signs = has_sign && !D.sign_at_store;
+    const int64_t ld = (PRO == PRO_CODES) ? D.ld_out : D.ld_in;   // same matrix either side
+    const unsigned ntiles = static_cast<unsigned>(D.ax[0].nt * D.ax[1].nt);
+    unsigned t = blockIdx.x;
+    if (t >= ntiles) return;
+    if (PRO == PRO_CODES && tid < 16) lev[tid] = Q.level[tid];
+    int *rloc = reinterpret_cast<int *>(sm + D.loc_base);   // tile-local part of each global index
+    int *cloc = rloc + Er;
+    for (int i = tid; i < Er; i += PT) rloc[i] = axis_global(D.ax[0], 0u, i);
+    for (int i = tid; i < Ec; i += PT) cloc[i] = axis_global(D.ax[1], 0u, i);
+    __syncthreads();
+
+    Pre R;
+    {
+        const Buf B0 = buf_of(sm, D, 0);
+        build_tables(D, B0, rloc, cloc, t, ld, tid);
+        __syncthreads();
+        load_pre<PRO>(D, Q, B0.tb, R, tid, warp, lane);
+        issue_coefs(D, B0.tb, B0.C, warp, lane);
+        cp_async_commit();
+        store_pre<PRO>(D, Q, B0.tb, T, B0.ssc, lev, R, load_signs, tid, warp, lane);
+        cp_async_wait_all();
+        __syncthreads();
+    }
+
+    for (int k = 0; t < ntiles; ++k, t += gridDim.x) {
+        const Buf B = buf_of(sm, D, k & 1);
+        const unsigned tn = t + gridDim.x;
+        const bool more = tn < ntiles;
+        const Buf Bn = buf_of(sm, D, (k + 1) & 1);
+        if (more) {
+            build_tables(D, Bn, rloc, cloc, tn, ld, tid);
+            __syncthreads();
+            load_pre<PRO>(D, Q, Bn.tb, R, tid, warp, lane);
+            issue_coefs(D, Bn.tb, Bn.C, warp, lane);
+            cp_async_commit();
+        }
+
+        for (int u = 0; u < D.nst; ++u) {
+            const PStage &S = D.st[u];
+            const bool rows = (S.axis == 0);
+            const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
+            if (S.kp == 8) stage_run<8, false>(T, B.C, S, A, Bv, NV, warp, lane);
+            else if (S.kp == 16) stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
+            else stage_rounds(T, B.C, S, A, Bv, NV, warp, lane);
             __syncthreads();
         }
-    } else {
-        if (Q.bits == 2) decode_tile<2>(T, D, Q, cw, ssc, lev, warp, lane);
-        else if (Q.bits == 3) decode_tile<3>(T, D, Q, cw, ssc, lev, warp, lane);
-        else decode_tile<4>(T, D, Q, cw, ssc, lev, warp, lane);
-        __syncthreads();
-    }
 
-    // the stages
-    for (int u = 0; u < D.nst; ++u) {
-        const PStage &S = D.st[u];
-        const bool rows = (S.axis == 0);
-        const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
-        if (S.kp == 8) stage_run<8, false>(T, C, S, A, Bv, NV, warp, lane);
-        else if (S.kp == 16) stage_run<16, false>(T, C, S, A, Bv, NV, warp, lane);
-        else stage_run<8, true>(T, C, S, A, Bv, NV, warp, lane);
+        if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
+            constexpr bool F = (EPI == EPI_QUANT_F32);
+            if (Q.bits == 2) quantize_tile_fast<2, F>(T, D, Q, B.tb, warp, lane);
+            else if (Q.bits == 4) quantize_tile_fast<4, F>(T, D, Q, B.tb, warp, lane);
+            else quantize_tile<3, F>(T, D, Q, B.tb, warp, lane);
+        } else {
+            store_tile<EPI>(T, D, B.tb, D.sign_at_store && has_sign, warp, lane);
+        }
         __syncthreads();
-    }
 
-    // epilogue
-    if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
-        constexpr bool F = (EPI == EPI_QUANT_F32);
-        if (Q.bits == 2) quantize_tile<2, F>(T, D, Q, rtab, ctab, warp, lane);
-        else if (Q.bits == 3) quantize_tile<3, F>(T, D, Q, rtab, ctab, warp, lane);
-        else quantize_tile<4, F>(T, D, Q, rtab, ctab, warp, lane);
-    } else {
-        const bool sg = D.sign_at_store && (D.ax[0].sign || D.ax[1].sign);
-        for (int tr = warp; tr < Er; tr += PW) {
-            const int64_t ro = static_cast<int64_t>(rtab[tr]) * D.ld_out;
-            const float rs = sg ? row_sign(D, rtab, tr) : 1.0f;
-            for (int tc = lane; tc < Ec; tc += 32) {
-                float v = T[tr * TCp + tc];
-                if (sg) v *= rs * col_sign(D, ctab, tc);
-                if constexpr (EPI == EPI_BF16)
-                    static_cast<__nv_bfloat16 *>(D.out)[ro + ctab[tc]] = __float2bfloat16_rn(v);
-                else
-                    static_cast<float *>(D.out)[ro + ctab[tc]] = v;
-            }
+        if (more) {
+            store_pre<PRO>(D, Q, Bn.tb, T, Bn.ssc, lev, R, load_signs, tid, warp, lane);
+            cp_async_wait_all();
+            __syncthreads();
         }
     }
 }
@@ -505,7 +885,7 @@ int pick_lv(int G, int NV) {
     double bu = -1.0;
     for (int lv = 32; lv >= 1; lv >>= 1) {
         const int lg = 32 / lv;
-        const int64_t vs = static_cast<int64_t>(lv) * 4 * ((NV + lv * 4 - 1) / (lv * 4));
+        const int64_t vs = static_cast<int64_t>(lv) * VL * ((NV + lv * VL - 1) / (lv * VL));
         const int64_t gs = static_cast<int64_t>(lg) * ((G + lg - 1) / lg);
         const double u = static_cast<double>(NV) / vs * static_cast<double>(G) / gs;
         if (u > bu + 1e-9) { bu = u; best = lv; }
@@ -539,20 +919,32 @@ int tcp_of(int Ec) { return (Ec % 2 == 0) ? Ec + 1 : Ec; }
 
 // Shared-memory bytes of a tile (layout of PassDesc: tile, coefficients,
 // tables, code staging).
-int64_t tile_smem(const PlanInput &in, int iL, int jL, int iR, int jR, int Er, int Ec, bool codes_stage) {
-    int64_t f = (static_cast<int64_t>(Er) * tcp_of(Ec) + 3) & ~int64_t(3);
-    if (in.L) f += stage_coef_floats(in.L, iL, jL, Er);
-    f += stage_coef_floats(in.R, iR, jR, Ec);
-    f += Er + Ec;
-    if (codes_stage) f += 16 + ((static_cast<int64_t>(Er) * (Ec / in.group) + 3) & ~int64_t(3)) +
-                          static_cast<int64_t>(Er) * Ec * 4 / 32;
-    return f * 4;
+// Shared memory of a pass kernel, in floats: the tile (odd pitch), then
+// two buffers of block coefficients + index tables (one for the tile being
+// computed, one for the next), the tile-local index tables, then 16
+// dequantised levels.
+struct SmemLayout {
+    int tile_floats, coef_floats, tab_base, buf_floats, loc_base, lev_base, total_floats;
+};
+
+SmemLayout smem_layout(const PlanInput &in, int iL, int jL, int iR, int jR, int Er, int Ec) {
+    SmemLayout L;
+    L.tile_floats = (Er * tcp_of(Ec) + 3) & ~3;
+    L.coef_floats = (in.L ? stage_coef_floats(in.L, iL, jL, Er) : 0) + stage_coef_floats(in.R, iR, jR, Ec);
+    L.tab_base = (L.coef_floats + 1) & ~1;
+    int b = L.tab_base + 2 * Er + 2 * Er + Er + 3 * Ec + Er + Ec;   // rin, rout (int64), rtab, ctab, cin, cout, signs
+    if (Ec % in.group == 0) b += Er * (Ec / in.group);            // scales of a codes tile
+    L.buf_floats = (b + 3) & ~3;
+    L.loc_base = L.tile_floats + 2 * L.buf_floats;
+    L.lev_base = L.loc_base + ((Er + Ec + 3) & ~3);
+    L.total_floats = L.lev_base + 16;
+    return L;
 }
 
 // Best tile for a pass applying L[iL:jL] and R[iR:jR]; `last` passes
 // quantise (forward) / decode codes (inverse) and need whole groups of
 // contiguous columns; `first` passes may read bf16 pairs.
-Cand best_tile(const PlanInput &in, int iL, int jL, int iR, int jR, bool first, bool last) {
+Cand best_tile(const PlanInput &in, int iL, int jL, int iR, int jR, bool first, bool last, int user_run) {
     Cand best;
     const AxisGeo gl = axis_geo(in.L, iL, jL), gr = axis_geo(in.R, iR, jR);
     const bool hasL = in.L && jL > iL, hasR = jR > iR;
@@ -568,11 +960,14 @@ Cand best_tile(const PlanInput &in, int iL, int jL, int iR, int jR, bool first, 
             const int64_t Ec = static_cast<int64_t>(gr.P) * XR;
             if (Er * Ec > TILE_MAX) break;
             const int64_t run = (gr.S > 1) ? XR : Ec;       // contiguous columns in memory
-            if (run % 2) continue;                          // bf16 pairs, 8-byte f32 pairs
+            if (run % 4 || Ec % 4) continue;                // 16-byte f32 / 8-byte bf16 quads
+            if (first && run < user_run) continue;          // the pass that reads (writes) the user matrix
             if (last && (Ec % in.group || Ec % 32)) continue;
-            if (first && Ec > 2 * 32 * MAXQ) continue;
-            if (tile_smem(in, iL, jL, iR, jR, static_cast<int>(Er), static_cast<int>(Ec), last) > SMEM_BUDGET)
+            if (last && Ec > 32 * MAXCH) continue;          // codes decode holds a row's chunks in registers
+            if (smem_layout(in, iL, jL, iR, jR, static_cast<int>(Er), static_cast<int>(Ec)).total_floats * 4 >
+                SMEM_BUDGET)
                 continue;
+            if (Er * Ec > NQR * 4 * PT) continue;           // register prefetch holds a whole tile
             int64_t nv = TILE_MAX;
             if (hasL) nv = std::min<int64_t>(nv, Ec);
             if (hasR) nv = std::min<int64_t>(nv, Er);
@@ -596,7 +991,7 @@ struct PassSpec {
 // Fewest passes (then best summed tile score) that take both processors
 // from stage 0 to the end; each pass takes a run of the next stages of
 // either side (at most MAXPS in all).
-bool plan_passes(const PlanInput &in, std::vector<PassSpec> &out) {
+bool plan_passes_run(const PlanInput &in, int user_run, std::vector<PassSpec> &out) {
     const int mL = in.L ? in.L->m : 0, mR = in.R->m;
     const int W = mR + 1;
     const int NS = (mL + 1) * W;
@@ -617,7 +1012,7 @@ bool plan_passes(const PlanInput &in, std::vector<PassSpec> &out) {
                     const int nid = jL * W + jR;
                     if (npass[nid] >= INF) continue;
                     const bool last = (jL == mL && jR == mR);
-                    const Cand c = best_tile(in, iL, jL, iR, jR, iL == 0 && iR == 0, last);
+                    const Cand c = best_tile(in, iL, jL, iR, jR, iL == 0 && iR == 0, last, user_run);
                     if (!c.ok) continue;
                     const int np = npass[nid] + 1;
                     const double sc = score[nid] + c.score;
@@ -640,6 +1035,14 @@ bool plan_passes(const PlanInput &in, std::vector<PassSpec> &out) {
     return true;
 }
 
+// The user matrix is read (forward) and written (inverse) by the first
+// forward pass; its rows are read in runs of at least 16 elements when some
+// plan allows it (shorter runs waste most of every 32-byte sector).
+bool plan_passes(const PlanInput &in, std::vector<PassSpec> &out) {
+    if (in.rows * in.cols >= (int64_t(1) << 31)) return false;
+    return plan_passes_run(in, 16, out) || plan_passes_run(in, 4, out);
+}
+
 void fill_axis(PAxis &A, const PlanDev *pl, int i, int j, int X, int64_t n) {
     const AxisGeo g = axis_geo(pl, i, j);
     A.n = n;
@@ -650,6 +1053,11 @@ void fill_axis(PAxis &A, const PlanDev *pl, int i, int j, int X, int64_t n) {
     A.nlo = g.S / A.Lx;
     A.nt = (n / (static_cast<int64_t>(A.P) * g.S * A.Hx)) * A.nlo;
     A.sign = nullptr;
+    A.f_nlo = make_fdiv(static_cast<unsigned>(A.nlo));
+    A.f_PS = make_fdiv(static_cast<unsigned>(A.P * A.S));
+    A.f_S = make_fdiv(static_cast<unsigned>(A.S));
+    A.f_Hx = make_fdiv(static_cast<unsigned>(A.Hx));
+    A.f_Lx = make_fdiv(static_cast<unsigned>(A.Lx));
 }
 
 // Stage descriptors of a pass: forward applies L[iL..jL) then R[iR..jR) in
@@ -695,17 +1103,22 @@ void fill_stages(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inve
 template <int PRO, int EPI>
 int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     static int attr_done[64] = {};
+    static int nsm[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && attr_done[dev] < D.smem_bytes) {
-        const cudaError_t e = cudaFuncSetAttribute(pass_kernel<PRO, EPI>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BUDGET);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(pass_kernel<PRO, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SMEM_BUDGET);
         if (e != cudaSuccess) return e;
-        attr_done[dev] = SMEM_BUDGET;
+        e = cudaDeviceGetAttribute(&nsm[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = 1;
     }
     const int64_t nb = D.ax[0].nt * D.ax[1].nt;
     if (nb <= 0) return 0;
-    pass_kernel<PRO, EPI><<<static_cast<unsigned>(nb), PT, D.smem_bytes, st>>>(D, Q);
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(nb, nsm[dev]));
+    pass_kernel<PRO, EPI><<<grid, PT, D.smem_bytes, st>>>(D, Q);
     return cudaGetLastError();
 }
 
@@ -726,35 +1139,97 @@ int dispatch(const PassDesc &D, const QuantDev &Q, int pro, int epi, cudaStream_
 
 // Build the descriptor of pass k of a plan (geometry, stages, shared-memory
 // layout); prologue/epilogue pointers are filled by the caller.
-void build_desc(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inverse, bool codes_stage) {
+void build_desc(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inverse) {
     D = PassDesc{};
     fill_axis(D.ax[0], in.L, ps.iL, ps.jL, ps.XL, in.rows);
     fill_axis(D.ax[1], in.R, ps.iR, ps.jR, ps.XR, in.cols);
     int cf = 0;
     fill_stages(D, in, ps, inverse, cf);
     D.TCp = tcp_of(D.ax[1].E);
-    D.coef_base = (D.ax[0].E * D.TCp + 3) & ~3;
+    const SmemLayout L = smem_layout(in, ps.iL, ps.jL, ps.iR, ps.jR, D.ax[0].E, D.ax[1].E);
+    D.tile_floats = L.tile_floats;
+    D.coef_base = 0;
     D.coef_floats = cf;
-    D.tab_base = D.coef_base + cf;
-    D.stage_base = D.tab_base + D.ax[0].E + D.ax[1].E;
-    int64_t total = D.stage_base;
-    if (codes_stage)
-        total += 16 + ((static_cast<int64_t>(D.ax[0].E) * (D.ax[1].E / in.group) + 3) & ~int64_t(3)) +
-                 static_cast<int64_t>(D.ax[0].E) * D.ax[1].E * 4 / 32;
-    D.smem_bytes = static_cast<int>(total * 4);
+    D.tab_base = L.tab_base;
+    D.buf_floats = L.buf_floats;
+    D.lev_base = L.lev_base;
+    D.loc_base = L.loc_base;
+    D.f_nch = make_fdiv(static_cast<unsigned>((D.ax[1].E + 31) / 32));
+    D.smem_bytes = L.total_floats * 4;
     if (in.L && ps.iL == 0 && ps.jL > 0) D.ax[0].sign = in.L->signs;
     if (ps.iR == 0 && ps.jR > 0) D.ax[1].sign = in.R->signs;
     D.sign_at_store = inverse ? 1 : 0;
     D.cols = in.cols;
 }
 
+thread_local void *const *t_events = nullptr;
+thread_local int t_nev = 0;
+
+void record_event(int k, cudaStream_t st) {
+    if (k < t_nev && t_events[k]) cudaEventRecord(static_cast<cudaEvent_t>(t_events[k]), st);
+}
+
 }  // namespace
+
+void set_pass_events(void *const *events, int n) {
+    t_events = (n > 0) ? events : nullptr;
+    t_nev = (n > 0) ? n : 0;
+}
 
 bool pass_plan_ok(const PlanDev &left, const PlanDev &right, int group) {
     PlanInput in{&left, &right, left.d, right.d, group};
     std::vector<PassSpec> ps;
     return plan_passes(in, ps);
 }
+
+int pass_count(const PlanDev &left, const PlanDev &right, int group) {
+    PlanInput in{&left, &right, left.d, right.d, group};
+    std::vector<PassSpec> ps;
+    return plan_passes(in, ps) ? static_cast<int>(ps.size()) : 0;
+}
+
+int pass_fma(const PlanDev &left, const PlanDev &right, int group, int k) {
+    PlanInput in{&left, &right, left.d, right.d, group};
+    std::vector<PassSpec> ps;
+    if (!plan_passes(in, ps) || k < 0 || k >= static_cast<int>(ps.size())) return -1;
+    int f = 0;
+    for (int t = ps[k].iL; t < ps[k].jL; ++t) f += left.st[t].b;
+    for (int t = ps[k].iR; t < ps[k].jR; ++t) f += right.st[t].b;
+    return f;
+}
+
+// Workspace buffers of a plan: the passes hand the matrix on through fp32
+// workspaces in the next pass's tile-major order, alternating between two
+// buffers of rows*cols floats (one when there are only two passes).
+namespace {
+
+void link_passes(PassDesc &D, const PlanInput &in, const std::vector<PassSpec> &ps, int k, bool inverse,
+                 float *ws, const void *user_in, void *user_out) {
+    const int np = static_cast<int>(ps.size());
+    const int64_t n = in.rows * in.cols;
+    D.ld_in = in.cols;
+    D.ld_out = in.cols;
+    if (k == 0) {
+        D.in = user_in;
+        D.in_blocked = 0;
+    } else {
+        D.in = ws + ((k - 1) % 2) * n;
+        D.in_blocked = 1;
+    }
+    if (k == np - 1) {
+        D.out = user_out;
+        D.out_blocked = 0;
+    } else {
+        D.out = ws + (k % 2) * n;
+        D.out_blocked = 1;
+        PassDesc Dn;
+        build_desc(Dn, in, ps[k + 1], inverse);
+        D.nx[0] = Dn.ax[0];
+        D.nx[1] = Dn.ax[1];
+    }
+}
+
+}  // namespace
 
 int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q, const void *in_ptr,
                     int in_dtype, uint8_t *codes, uint16_t *scales, float *rotated_out, float *ws,
@@ -764,29 +1239,23 @@ int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q
     if (!plan_passes(in, ps)) return cudaErrorInvalidValue;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int np = static_cast<int>(ps.size());
+    record_event(0, st);
     for (int k = 0; k < np; ++k) {
         const bool first = (k == 0), last = (k == np - 1);
         PassDesc D;
-        build_desc(D, in, ps[k], false, last);
+        build_desc(D, in, ps[k], false);
+        link_passes(D, in, ps, k, false, ws, in_ptr, nullptr);
         int pro = PRO_F32, epi = EPI_F32;
-        if (first) {
-            pro = (in_dtype == HARP_BF16) ? PRO_BF16 : PRO_F32;
-            D.in = in_ptr;
-        } else {
-            D.in = ws;
-        }
-        D.ld_in = in.cols;
+        if (first) pro = (in_dtype == HARP_BF16) ? PRO_BF16 : PRO_F32;
         if (last) {
             epi = rotated_out ? EPI_QUANT_F32 : EPI_QUANT;
             D.codes = codes;
             D.scales = scales;
             D.out_f32 = rotated_out;
-        } else {
-            D.out = ws;
-            D.ld_out = in.cols;
         }
         const int e = dispatch(D, q, pro, epi, st);
         if (e) return e;
+        record_event(k + 1, st);
     }
     return 0;
 }
@@ -799,28 +1268,22 @@ int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q
     std::reverse(ps.begin(), ps.end());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int np = static_cast<int>(ps.size());
+    record_event(0, st);
     for (int k = 0; k < np; ++k) {
         const bool first = (k == 0), last = (k == np - 1);
         PassDesc D;
-        build_desc(D, in, ps[k], true, first);
+        build_desc(D, in, ps[k], true);
+        link_passes(D, in, ps, k, true, ws, nullptr, out);
         int pro = PRO_F32, epi = EPI_F32;
         if (first) {
             pro = PRO_CODES;
             D.in_codes = codes;
             D.in_scales = scales;
-        } else {
-            D.in = ws;
-            D.ld_in = in.cols;
         }
-        D.ld_out = in.cols;
-        if (last) {
-            epi = (out_dtype == HARP_BF16) ? EPI_BF16 : EPI_F32;
-            D.out = out;
-        } else {
-            D.out = ws;
-        }
+        if (last) epi = (out_dtype == HARP_BF16) ? EPI_BF16 : EPI_F32;
         const int e = dispatch(D, q, pro, epi, st);
         if (e) return e;
+        record_event(k + 1, st);
     }
     return 0;
 }

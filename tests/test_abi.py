@@ -151,6 +151,12 @@ def test_compute_calls_reject_bad_arguments_before_launch():
     assert L.harp_quantize(cb.handle, ctypes.c_void_p(4100), 0, 1, 128, 128, fake, fake, None) == 4
     # leading dimension too small
     assert L.harp_quantize(cb.handle, fake, 0, 2, 128, 64, fake, fake, None) == 2
+    # timing hook and pass count argument checks
+    assert L.harp_set_pass_events(None, -1) == 1
+    assert L.harp_set_pass_events(None, 3) == 1
+    assert L.harp_set_pass_events(None, 0) == 0
+    assert L.harp_pass_count(None, None, None, None) == 1
+    assert L.harp_pass_fma(None, None, None, 0, None) == 1
     n = ctypes.c_size_t()
     assert L.harp_workspace_size(None, None, 10, 20, ctypes.byref(n)) == 0 and n.value == 0
-    assert L.harp_workspace_size(ctypes.c_void_p(8), None, 10, 20, ctypes.byref(n)) == 0 and n.value == 800
+    assert L.harp_workspace_size(ctypes.c_void_p(8), None, 10, 20, ctypes.byref(n)) == 0 and n.value == 1600

@@ -321,5 +321,32 @@ def test_plan_info_and_workspace():
     s = synth.side_draws(5, (43, 16, 16), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
     plan = harp.Plan.from_side(s)
     assert plan.info() == (11008, 3, (43, 16, 16))
-    assert harp.workspace_size(plan, plan, 11008, 11008) == 11008 * 11008 * 4
+    assert harp.workspace_size(plan, plan, 11008, 11008) == 11008 * 11008 * 8
     assert harp.workspace_size(None, plan, 7, 11008) == 0
+
+
+def test_pass_events_time_each_pass():
+    """harp_pass_count reports the pass kernels of the two-sided calls and
+    harp_set_pass_events gets one event per pass boundary recorded; results
+    do not change when events are registered."""
+    w = wl("c2")
+    q = w.quants[0]
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    n = harp.harp_pass_count(left, right, cb)
+    assert n >= 2
+    assert harp.harp_pass_count(None, right, cb) == 0
+    # every stage of both processors is applied by exactly one pass
+    assert sum(harp.harp_pass_fma(left, right, cb, k) for k in range(n)) == 2 * 48
+    x = to_dev(w)
+    codes, scales, _ = harp.rotate_quantize(left, right, cb, x)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    harp.harp_set_pass_events(evs)
+    try:
+        codes2, scales2, _ = harp.rotate_quantize(left, right, cb, x)
+    finally:
+        harp.harp_set_pass_events([])
+    torch.cuda.synchronize()
+    times = [evs[k].elapsed_time(evs[k + 1]) for k in range(n)]
+    assert all(t > 0 for t in times)
+    assert torch.equal(codes2, codes) and torch.equal(scales2, scales)

@@ -38,7 +38,7 @@ def _case(rows_radix, cols_radix, bits, group, seed):
 def test_static_workspace_matches_caller_workspace_twice():
     import torch
     torch.cuda.set_device(0)
-    # 1024 x 2048 two-sided: an 8 MiB intermediate, inside the 32 MiB array
+    # 1024 x 2048 two-sided: a 16 MiB workspace need, inside the 32 MiB array
     left, right, cb, x = _case((16, 8, 8), (16, 16, 8), 4, 128, 31)
     rows, cols = x.shape
     assert harp.workspace_size(left, right, rows, cols) <= harp.HARP_STATIC_WORKSPACE_BYTES
@@ -64,7 +64,7 @@ def test_static_workspace_matches_caller_workspace_twice():
 def test_static_workspace_rejects_oversized_matrix():
     import torch
     torch.cuda.set_device(0)
-    # 4096 x 4096 needs a 64 MiB intermediate: refused before any pointer is used
+    # 4096 x 4096 needs a 128 MiB workspace: refused before any pointer is used
     left, right, cb, _ = _case((16, 16, 16), (16, 16, 16), 2, 128, 5)
     assert harp.workspace_size(left, right, 4096, 4096) > harp.HARP_STATIC_WORKSPACE_BYTES
     dummy = ctypes.c_void_p(1 << 20)
