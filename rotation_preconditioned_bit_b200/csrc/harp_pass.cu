@@ -111,6 +111,9 @@ struct PassDesc {
     int lev_base;       // float offset of the 16 dequantised levels
     int loc_base;       // float offset of the per-pass local index tables (rows, then columns)
     FDiv f_nch;         // division by the number of 32-column chunks of a tile row
+    FDiv f_wpr;         // ... by the packed code words of a tile row
+    FDiv f_ngt;         // ... by the quantiser groups of a tile row
+    FDiv f_gch;         // ... by the 32-code chunks of a quantiser group
     int coef_base;      // float offset of the coefficient area
     int coef_floats;
     int tab_base;       // float offset of the index tables (rows, then cols)
@@ -227,35 +230,42 @@ __device__ __forceinline__ void unit_addr(const PStage &S, int gi, int v0, int L
 // into both halves). CLAMP: inputs past b are read at b-1 and meet zero
 // coefficients (only when b is not a multiple of 4).
 template <int K, bool CLAMP>
+__device__ __forceinline__ void unit_step(const float *T, const float *wrow, int j, int b, int step,
+                                          const int (&p)[VL], f2_t (&acc)[K / 2][VL]) {
+    const int off = (CLAMP ? min(j, b - 1) : j) * step;
+    f2_t x[VL];
+#pragma unroll
+    for (int v = 0; v < VL; ++v) {
+        const float xv = T[p[v] + off];
+        x[v] = f2_pack(xv, xv);
+    }
+    const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
+#pragma unroll
+    for (int q = 0; q < K / 4; ++q) {
+        const float4 w = w4[q];
+        const f2_t wa = f2_pack(w.x, w.y), wb = f2_pack(w.z, w.w);
+#pragma unroll
+        for (int v = 0; v < VL; ++v) {
+            acc[2 * q][v] = f2_fma(wa, x[v], acc[2 * q][v]);
+            acc[2 * q + 1][v] = f2_fma(wb, x[v], acc[2 * q + 1][v]);
+        }
+    }
+}
+
+// JP > 0: the block has exactly JP inputs and K outputs (fully unrolled).
+template <int K, bool CLAMP, int JP = 0>
 __device__ __forceinline__ void unit_compute(const float *T, const float *wp, int kp, int jpad, int b,
                                              int step, const int (&p)[VL], f2_t (&acc)[K / 2][VL]) {
 #pragma unroll
     for (int q = 0; q < K / 2; ++q)
 #pragma unroll
         for (int v = 0; v < VL; ++v) acc[q][v] = 0ull;
-    for (int j0 = 0; j0 < jpad; j0 += 4) {
+    if constexpr (JP > 0) {
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int j = j0 + jj;
-            const int off = (CLAMP ? min(j, b - 1) : j) * step;
-            f2_t x[VL];
-#pragma unroll
-            for (int v = 0; v < VL; ++v) {
-                const float xv = T[p[v] + off];
-                x[v] = f2_pack(xv, xv);
-            }
-            const float4 *w4 = reinterpret_cast<const float4 *>(wp + j * kp);
-#pragma unroll
-            for (int q = 0; q < K / 4; ++q) {
-                const float4 w = w4[q];
-                const f2_t wa = f2_pack(w.x, w.y), wb = f2_pack(w.z, w.w);
-#pragma unroll
-                for (int v = 0; v < VL; ++v) {
-                    acc[2 * q][v] = f2_fma(wa, x[v], acc[2 * q][v]);
-                    acc[2 * q + 1][v] = f2_fma(wb, x[v], acc[2 * q + 1][v]);
-                }
-            }
-        }
+        for (int j = 0; j < JP; ++j) unit_step<K, CLAMP>(T, wp + j * K, j, b, step, p, acc);
+    } else {
+#pragma unroll 4
+        for (int j = 0; j < jpad; ++j) unit_step<K, CLAMP>(T, wp + j * kp, j, b, step, p, acc);
     }
 }
 
@@ -473,13 +483,10 @@ __device__ __forceinline__ void store_tile(const float *T, const PassDesc &D, co
 // xor tree.
 template <int BITS, bool F32COPY>
 __device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDesc &D, const QuantDev &Q,
-                                                   const Tabs &tb, int warp, int lane) {
+                                                   const Tabs &tb, const float *ts, int warp, int lane) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     const int g = Q.group, ngt = Ec / g, nit = g >> 5;
     const bool is_max = (Q.kind == HARP_ABSMAX);
-    float t[(1 << BITS) - 1];
-#pragma unroll
-    for (int k = 0; k < (1 << BITS) - 1; ++k) t[k] = Q.thr[k];
     const int64_t spr = D.cols / g;
     const int64_t wpr = D.cols * BITS / 32;
     const int q = lane >> 2, c = lane & 3;
@@ -511,7 +518,7 @@ __device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDes
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 x[e] = rp[32 * it + e];
-                word |= static_cast<unsigned>(code_of<BITS>(x[e], s, inv, !is_max, t)) << (BITS * e);
+                word |= static_cast<unsigned>(code_of_smem<BITS>(x[e], s, inv, !is_max, ts)) << (BITS * e);
             }
             const int64_t col = c0 + 32 * it + 8 * c;       // first of this lane's 8 columns
             if constexpr (BITS == 4) {
@@ -643,7 +650,7 @@ __device__ __forceinline__ void decode_rows(const PassDesc &D, const QuantDev &Q
                 const unsigned w1 = (sh + BITS > 32) ? wsrc[ch * BITS + wi + 1] : 0u;
                 unsigned code = w0 >> sh;
                 if (sh + BITS > 32) code |= w1 << (32 - sh);
-                val[ch] = ssc[tr * ngt + (ch * 32) / Q.group] * lev[code & MASK];
+                val[ch] = ssc[tr * ngt + static_cast<int>(fdiv(static_cast<unsigned>(ch), D.f_gch))] * lev[code & MASK];
             }
         }
         __syncwarp();
@@ -679,13 +686,13 @@ __device__ __forceinline__ void load_pre(const PassDesc &D, const QuantDev &Q, c
             const int i = tid + PT * k;
             R.w[k] = 0u;
             if (i < Er * wpr) {
-                const int tr = i / wpr, w = i - tr * wpr;
+                const int tr = static_cast<int>(fdiv(static_cast<unsigned>(i), D.f_wpr)), w = i - tr * wpr;
                 R.w[k] = __ldg(words + static_cast<int64_t>(tb.rtab[tr]) * rw + (c0 >> 5) * Q.bits + w);
             }
         }
         R.sc = 0.0f;
         if (tid < Er * ngt) {
-            const int tr = tid / ngt, q = tid - tr * ngt;
+            const int tr = static_cast<int>(fdiv(static_cast<unsigned>(tid), D.f_ngt)), q = tid - tr * ngt;
             R.sc = __half2float(__ushort_as_half(
                 __ldg(D.in_scales + static_cast<int64_t>(tb.rtab[tr]) * (D.cols / Q.group) + c0 / Q.group + q)));
         }
@@ -725,7 +732,7 @@ __device__ __forceinline__ void store_pre(const PassDesc &D, const QuantDev &Q, 
         for (int k = 0; k < NWR; ++k) {
             const int i = tid + PT * k;
             if (i < Er * wpr) {
-                const int tr = i / wpr, w = i - tr * wpr;
+                const int tr = static_cast<int>(fdiv(static_cast<unsigned>(i), D.f_wpr)), w = i - tr * wpr;
                 reinterpret_cast<unsigned *>(T + tr * TCp + (Ec - wpr))[w] = R.w[k];
             }
         }
@@ -785,7 +792,10 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
     const unsigned ntiles = static_cast<unsigned>(D.ax[0].nt * D.ax[1].nt);
     unsigned t = blockIdx.x;
     if (t >= ntiles) return;
-    if (PRO == PRO_CODES && tid < 16) lev[tid] = Q.level[tid];
+    if (tid < 16) {
+        lev[tid] = Q.level[tid];
+        lev[16 + tid] = Q.thr[tid];     // midpoints (Lloyd-Max code search)
+    }
     int *rloc = reinterpret_cast<int *>(sm + D.loc_base);   // tile-local part of each global index
     int *cloc = rloc + Er;
     for (int i = tid; i < Er; i += PT) rloc[i] = axis_global(D.ax[0], 0u, i);
@@ -830,8 +840,8 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
 
         if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
             constexpr bool F = (EPI == EPI_QUANT_F32);
-            if (Q.bits == 2) quantize_tile_fast<2, F>(T, D, Q, B.tb, warp, lane);
-            else if (Q.bits == 4) quantize_tile_fast<4, F>(T, D, Q, B.tb, warp, lane);
+            if (Q.bits == 2) quantize_tile_fast<2, F>(T, D, Q, B.tb, lev + 16, warp, lane);
+            else if (Q.bits == 4) quantize_tile_fast<4, F>(T, D, Q, B.tb, lev + 16, warp, lane);
             else quantize_tile<3, F>(T, D, Q, B.tb, warp, lane);
         } else {
             store_tile<EPI>(T, D, B.tb, D.sign_at_store && has_sign, warp, lane);
@@ -904,6 +914,7 @@ struct PlanInput {
     const PlanDev *R;
     int64_t rows, cols;
     int group;
+    int bits;
 };
 
 int stage_coef_floats(const PlanDev *pl, int i, int j, int E) {
@@ -937,7 +948,7 @@ SmemLayout smem_layout(const PlanInput &in, int iL, int jL, int iR, int jR, int 
     L.buf_floats = (b + 3) & ~3;
     L.loc_base = L.tile_floats + 2 * L.buf_floats;
     L.lev_base = L.loc_base + ((Er + Ec + 3) & ~3);
-    L.total_floats = L.lev_base + 16;
+    L.total_floats = L.lev_base + 32;
     return L;
 }
 
@@ -1155,6 +1166,9 @@ void build_desc(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inver
     D.lev_base = L.lev_base;
     D.loc_base = L.loc_base;
     D.f_nch = make_fdiv(static_cast<unsigned>((D.ax[1].E + 31) / 32));
+    D.f_wpr = make_fdiv(static_cast<unsigned>(std::max(1, (D.ax[1].E / 32) * in.bits)));
+    D.f_ngt = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / in.group)));
+    D.f_gch = make_fdiv(static_cast<unsigned>(std::max(1, in.group / 32)));
     D.smem_bytes = L.total_floats * 4;
     if (in.L && ps.iL == 0 && ps.jL > 0) D.ax[0].sign = in.L->signs;
     if (ps.iR == 0 && ps.jR > 0) D.ax[1].sign = in.R->signs;
@@ -1177,19 +1191,19 @@ void set_pass_events(void *const *events, int n) {
 }
 
 bool pass_plan_ok(const PlanDev &left, const PlanDev &right, int group) {
-    PlanInput in{&left, &right, left.d, right.d, group};
+    PlanInput in{&left, &right, left.d, right.d, group, 4};
     std::vector<PassSpec> ps;
     return plan_passes(in, ps);
 }
 
 int pass_count(const PlanDev &left, const PlanDev &right, int group) {
-    PlanInput in{&left, &right, left.d, right.d, group};
+    PlanInput in{&left, &right, left.d, right.d, group, 4};
     std::vector<PassSpec> ps;
     return plan_passes(in, ps) ? static_cast<int>(ps.size()) : 0;
 }
 
 int pass_fma(const PlanDev &left, const PlanDev &right, int group, int k) {
-    PlanInput in{&left, &right, left.d, right.d, group};
+    PlanInput in{&left, &right, left.d, right.d, group, 4};
     std::vector<PassSpec> ps;
     if (!plan_passes(in, ps) || k < 0 || k >= static_cast<int>(ps.size())) return -1;
     int f = 0;
@@ -1234,7 +1248,7 @@ void link_passes(PassDesc &D, const PlanInput &in, const std::vector<PassSpec> &
 int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q, const void *in_ptr,
                     int in_dtype, uint8_t *codes, uint16_t *scales, float *rotated_out, float *ws,
                     void *stream) {
-    PlanInput in{&left, &right, left.d, right.d, q.group};
+    PlanInput in{&left, &right, left.d, right.d, q.group, q.bits};
     std::vector<PassSpec> ps;
     if (!plan_passes(in, ps)) return cudaErrorInvalidValue;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1262,7 +1276,7 @@ int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q
 
 int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q, const uint8_t *codes,
                     const uint16_t *scales, void *out, int out_dtype, float *ws, void *stream) {
-    PlanInput in{&left, &right, left.d, right.d, q.group};
+    PlanInput in{&left, &right, left.d, right.d, q.group, q.bits};
     std::vector<PassSpec> ps;
     if (!plan_passes(in, ps)) return cudaErrorInvalidValue;
     std::reverse(ps.begin(), ps.end());

@@ -75,6 +75,23 @@ __device__ __forceinline__ int code_of(float x, float s, float inv_s, bool lloyd
     return static_cast<int>(fminf(fmaxf(rintf(z), -qmax), qmax)) + HALF;
 }
 
+// The same code with the midpoints in shared memory (ts[k], k < 2^BITS - 1):
+// a binary search of BITS dependent steps, each one load and one compare.
+template <int BITS>
+__device__ __forceinline__ int code_of_smem(float x, float s, float inv_s, bool lloyd, const float *ts) {
+    constexpr int HALF = 1 << (BITS - 1);
+    if (!(s > 0.0f)) return HALF;
+    const float z = x * inv_s;
+    if (lloyd) {
+        int code = 0;
+#pragma unroll
+        for (int step = HALF; step >= 1; step >>= 1) code += (z > ts[code + step - 1]) ? step : 0;
+        return code;
+    }
+    const float qmax = static_cast<float>(HALF - 1);
+    return static_cast<int>(fminf(fmaxf(rintf(z), -qmax), qmax)) + HALF;
+}
+
 template <int BITS>
 __device__ __forceinline__ unsigned pack_words(int code, int lane) {
     const int bit0 = BITS * lane;
