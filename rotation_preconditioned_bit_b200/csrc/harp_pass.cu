@@ -225,47 +225,42 @@ __device__ __forceinline__ void unit_addr(const PStage &S, int gi, int v0, int L
 }
 
 // acc[q][v] = (out 2q, out 2q+1) of vector v: sum_j w[j][k] * x_v[j] for K
-// outputs and VL vectors, as packed pairs of outputs (the coefficient row
-// w[j][0..K) is read as K/4 16-byte words = K/2 pairs; x_v[j] is broadcast
-// into both halves). CLAMP: inputs past b are read at b-1 and meet zero
-// coefficients (only when b is not a multiple of 4).
+// outputs and VL vectors, as packed pairs of outputs: the coefficient row
+// w[j][0..K) is read as K/4 16-byte words, each two ready-made pairs, and
+// x_v[j] is broadcast into both halves. CLAMP: inputs past b are read at b-1
+// and meet zero coefficients (only when b is not a multiple of 4).
 template <int K, bool CLAMP>
-__device__ __forceinline__ void unit_step(const float *T, const float *wrow, int j, int b, int step,
-                                          const int (&p)[VL], f2_t (&acc)[K / 2][VL]) {
-    const int off = (CLAMP ? min(j, b - 1) : j) * step;
-    f2_t x[VL];
-#pragma unroll
-    for (int v = 0; v < VL; ++v) {
-        const float xv = T[p[v] + off];
-        x[v] = f2_pack(xv, xv);
-    }
-    const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
-#pragma unroll
-    for (int q = 0; q < K / 4; ++q) {
-        const float4 w = w4[q];
-        const f2_t wa = f2_pack(w.x, w.y), wb = f2_pack(w.z, w.w);
-#pragma unroll
-        for (int v = 0; v < VL; ++v) {
-            acc[2 * q][v] = f2_fma(wa, x[v], acc[2 * q][v]);
-            acc[2 * q + 1][v] = f2_fma(wb, x[v], acc[2 * q + 1][v]);
-        }
-    }
-}
-
-// JP > 0: the block has exactly JP inputs and K outputs (fully unrolled).
-template <int K, bool CLAMP, int JP = 0>
 __device__ __forceinline__ void unit_compute(const float *T, const float *wp, int kp, int jpad, int b,
                                              int step, const int (&p)[VL], f2_t (&acc)[K / 2][VL]) {
 #pragma unroll
     for (int q = 0; q < K / 2; ++q)
 #pragma unroll
         for (int v = 0; v < VL; ++v) acc[q][v] = 0ull;
-    if constexpr (JP > 0) {
+    const float *xp[VL];
 #pragma unroll
-        for (int j = 0; j < JP; ++j) unit_step<K, CLAMP>(T, wp + j * K, j, b, step, p, acc);
-    } else {
+    for (int v = 0; v < VL; ++v) xp[v] = T + p[v];
+    const ulonglong2 *wq = reinterpret_cast<const ulonglong2 *>(wp);
+    const int wstep = kp / 4;      // 16-byte words per coefficient row
+    const int jlast = (b - 1) * step;
 #pragma unroll 4
-        for (int j = 0; j < jpad; ++j) unit_step<K, CLAMP>(T, wp + j * kp, j, b, step, p, acc);
+    for (int j = 0; j < jpad; ++j) {
+        f2_t x[VL];
+#pragma unroll
+        for (int v = 0; v < VL; ++v) {
+            const float xv = CLAMP ? xp[v][min(j * step, jlast)] : *xp[v];
+            x[v] = f2_pack(xv, xv);
+            if (!CLAMP) xp[v] += step;
+        }
+#pragma unroll
+        for (int q = 0; q < K / 4; ++q) {
+            const ulonglong2 w = wq[q];
+#pragma unroll
+            for (int v = 0; v < VL; ++v) {
+                acc[2 * q][v] = f2_fma(w.x, x[v], acc[2 * q][v]);
+                acc[2 * q + 1][v] = f2_fma(w.y, x[v], acc[2 * q + 1][v]);
+            }
+        }
+        wq += wstep;
     }
 }
 
