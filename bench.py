@@ -281,6 +281,64 @@ def run_gpu(args, rank, world, local_rank):
     return total_ms, step_ms, kt, clk, e2e, npass, pass_fma
 
 
+def run_workloads(steps, dev):
+    """The other synthetic workloads, through the public calls with inputs
+    resident on the device: per call, mean device time over `steps` calls
+    (CUDA events; L2 not flushed: each call streams more than L2 except c1),
+    algorithmic GB/s (input read + codes + scales written for a forward;
+    codes + scales read + output written for an inverse) and elements/s."""
+    import numpy as np
+    import torch
+
+    import rotation_preconditioned_bit_b200 as harp
+    from rotation_preconditioned_bit_b200 import synth
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps * 1e-3
+
+    out = {}
+    for name in ("c1", "c3", "c4", "c5"):
+        w = synth.workload(name)
+        rows, cols = w.rows, w.cols
+        if w.dtype == "bf16":
+            x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).to(dev)
+            in_b = 2
+        else:
+            x = torch.from_numpy(w.x).to(dev)
+            in_b = 4
+        right = harp.Plan.from_side(w.right)
+        left = harp.Plan.from_side(w.left) if w.left is not None else None
+        ws = harp.empty_workspace(left, right, rows, cols, dev) if left else None
+        for q in w.quants:
+            cb = harp.Codebook(q.kind, q.bits, q.group)
+            codes, scales = harp.empty_codes(rows, cols, cb, dev)
+            code_b = q.bits / 8.0 + 2.0 / q.group
+            n = rows * cols
+            key = f"{w.name}_{q.kind}{q.bits}_g{q.group}"
+            t = timed(lambda: harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws))
+            rec = {"shape": [rows, cols], "fwd_us": round(t * 1e6, 2),
+                   "fwd_gbs": round(n * (in_b + code_b) / t / 1e9, 2), "fwd_elems_per_s": float(f"{n / t:.4g}")}
+            if left is not None:
+                o = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+                t = timed(lambda: harp.harp_dequantize_unrotate(left, right, cb, codes, scales, o, ws))
+                rec.update({"inv_us": round(t * 1e6, 2), "inv_gbs": round(n * (2 + code_b) / t / 1e9, 2),
+                            "inv_elems_per_s": float(f"{n / t:.4g}")})
+                rec["passes"] = harp.harp_pass_count(left, right, cb)
+            out[key] = rec
+        del x, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def kernel_table(kt, npass, pass_fma):
     """Per pass kernel: mean duration, the bytes it moves itself (input read,
     output written: bf16 weight, fp32 workspace, codes + scales), the
@@ -402,6 +460,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--workloads", action="store_true",
+                    help="also time the c1, c3, c4 and c5 workloads (adds ~1 min of input generation)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -441,6 +501,8 @@ def main():
             dt, credited, desc = oracle_sample(frac)
             cpu = {"value": round(credited / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                    "sample": desc, "seconds": round(dt, 2)}
+        wl = (run_workloads(max(3, args.steps // 4), torch.device("cuda", local_rank))
+              if args.workloads and world == 1 else None)
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
@@ -453,6 +515,8 @@ def main():
                 "hbm_frac": round(value / world / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": peak_src,
                 "roofline": roof, "kernels": ktab, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 2 * len(BITS) * npass * args.steps, "clocks": clk}
+        if wl is not None:
+            line["workloads"] = wl
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()
