@@ -114,6 +114,9 @@ struct PassDesc {
     FDiv f_wpr;         // ... by the packed code words of a tile row
     FDiv f_ngt;         // ... by the quantiser groups of a tile row
     FDiv f_gch;         // ... by the 32-code chunks of a quantiser group
+    FDiv f_nq;          // ... by the column quads of a tile row
+    FDiv f_nchc;        // ... by the 32-column chunks of a tile row (codes)
+    int stage_base;     // float offset of the staging buffer of the next tile's input
     int coef_base;      // float offset of the coefficient area
     int coef_floats;
     int tab_base;       // float offset of the index tables (rows, then cols)
@@ -624,146 +627,113 @@ __device__ __forceinline__ void issue_coefs(const PassDesc &D, const Tabs &tb, f
     }
 }
 
-constexpr int MAXCH = 8;   // 32-code chunks per tile row for the codes input (Ec <= 256)
+constexpr int MAXCH = 8;   // 32-code chunks per row of a quantised tile (Ec <= 256)
 
-template <int BITS>
-__device__ __forceinline__ void decode_rows(const PassDesc &D, const QuantDev &Q, float *T, const float *ssc,
-                                            const float *lev, int warp, int lane) {
-    constexpr unsigned MASK = (1u << BITS) - 1u;
-    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
-    const int nch = Ec >> 5, wpr = nch * BITS, ngt = Ec / Q.group;
-    const int bit = lane * BITS, wi = bit >> 5, sh = bit & 31;
-    for (int tr = warp; tr < Er; tr += PW) {
-        float *row = T + tr * TCp;
-        const unsigned *wsrc = reinterpret_cast<const unsigned *>(row + (Ec - wpr));
-        float val[MAXCH];
-#pragma unroll
-        for (int ch = 0; ch < MAXCH; ++ch) {
-            val[ch] = 0.0f;
-            if (ch < nch) {
-                const unsigned w0 = wsrc[ch * BITS + wi];
-                const unsigned w1 = (sh + BITS > 32) ? wsrc[ch * BITS + wi + 1] : 0u;
-                unsigned code = w0 >> sh;
-                if (sh + BITS > 32) code |= w1 << (32 - sh);
-                val[ch] = ssc[tr * ngt + static_cast<int>(fdiv(static_cast<unsigned>(ch), D.f_gch))] * lev[code & MASK];
-            }
-        }
-        __syncwarp();
-#pragma unroll
-        for (int ch = 0; ch < MAXCH; ++ch)
-            if (ch < nch) row[ch * 32 + lane] = val[ch];
-    }
+
+// The next tile's input is copied asynchronously into a dense staging
+// buffer (row-major [Er][Ec] fp32 or bf16, or the tile rows' packed code
+// words) while the current tile is computed; its scales (codes input) travel
+// in one register per thread.
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem));
 }
 
-// The next tile's input travels in registers while the current tile is
-// computed: per thread NQR quads of 4 values (16 bytes of fp32, 8 of bf16),
-// or for packed codes NWR words and one scale.
-constexpr int NQR = 8;    // quads per thread: 16K-element tiles / 512 threads / 4
-constexpr int NWR = 4;    // code words per thread: 16K codes * 4 bits / 32 / 512
-
-struct Pre {
-    uint4 q[NQR];
-    unsigned w[NWR];
-    float sc;
-};
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(gmem));
+}
 
 template <int PRO>
-__device__ __forceinline__ void load_pre(const PassDesc &D, const QuantDev &Q, const Tabs &tb, Pre &R, int tid,
-                                         int warp, int lane) {
+__device__ __forceinline__ float issue_input(const PassDesc &D, const QuantDev &Q, const Tabs &tb, void *S, int tid) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E;
+    float sc = 0.0f;
     if constexpr (PRO == PRO_CODES) {
         const int wpr = (Ec >> 5) * Q.bits, ngt = Ec / Q.group;
         const int64_t rw = D.cols * Q.bits / 32;
         const uint32_t *words = reinterpret_cast<const uint32_t *>(D.in_codes);
         const int c0 = tb.ctab[0];
-#pragma unroll
-        for (int k = 0; k < NWR; ++k) {
-            const int i = tid + PT * k;
-            R.w[k] = 0u;
-            if (i < Er * wpr) {
-                const int tr = static_cast<int>(fdiv(static_cast<unsigned>(i), D.f_wpr)), w = i - tr * wpr;
-                R.w[k] = __ldg(words + static_cast<int64_t>(tb.rtab[tr]) * rw + (c0 >> 5) * Q.bits + w);
-            }
+        for (int i = tid; i < Er * wpr; i += PT) {
+            const int tr = static_cast<int>(fdiv(static_cast<unsigned>(i), D.f_wpr)), w = i - tr * wpr;
+            cp_async4(static_cast<uint32_t *>(S) + tr * wpr + w,
+                      words + static_cast<int64_t>(tb.rtab[tr]) * rw + (c0 >> 5) * Q.bits + w);
         }
-        R.sc = 0.0f;
         if (tid < Er * ngt) {
             const int tr = static_cast<int>(fdiv(static_cast<unsigned>(tid), D.f_ngt)), q = tid - tr * ngt;
-            R.sc = __half2float(__ushort_as_half(
+            sc = __half2float(__ushort_as_half(
                 __ldg(D.in_scales + static_cast<int64_t>(tb.rtab[tr]) * (D.cols / Q.group) + c0 / Q.group + q)));
         }
     } else {
-        const int nch = (Ec + 31) >> 5, nu = ((Er + 3) >> 2) * nch;
-#pragma unroll
-        for (int k = 0; k < NQR; ++k) {
-            const int u = warp + PW * k;
-            const Quad qd = quad_of(u, D.f_nch, Er, Ec, lane);
-            R.q[k] = make_uint4(0u, 0u, 0u, 0u);
-            if (u < nu && qd.ok) {
-                const int64_t off = tb.rin[qd.tr] + tb.cin[qd.tc];
-                if constexpr (PRO == PRO_F32) {
-                    R.q[k] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(D.in) + off));
-                } else {
-                    const uint2 t = __ldg(reinterpret_cast<const uint2 *>(
-                        static_cast<const unsigned short *>(D.in) + off));
-                    R.q[k].x = t.x;
-                    R.q[k].y = t.y;
-                }
-            }
+        const int nq = Er * (Ec >> 2);                  // quads of 4 consecutive tile columns
+        const int nqr = Ec >> 2;
+        for (int i = tid; i < nq; i += PT) {
+            const int tr = static_cast<int>(fdiv(static_cast<unsigned>(i), D.f_nq)), tc = 4 * (i - tr * nqr);
+            const int64_t off = tb.rin[tr] + tb.cin[tc];
+            if constexpr (PRO == PRO_F32)
+                cp_async16(static_cast<float *>(S) + tr * Ec + tc, static_cast<const float *>(D.in) + off);
+            else
+                cp_async8(static_cast<unsigned short *>(S) + tr * Ec + tc,
+                          static_cast<const unsigned short *>(D.in) + off);
         }
+    }
+    return sc;
+}
+
+// Staging buffer -> fp32 tile (forward sign factors when asked; codes are
+// decoded with their group scales).
+template <int BITS>
+__device__ __forceinline__ void decode_staged(const PassDesc &D, const QuantDev &Q, const uint32_t *S, float *T,
+                                              const float *ssc, const float *lev, int warp, int lane) {
+    constexpr unsigned MASK = (1u << BITS) - 1u;
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
+    const int nch = Ec >> 5, wpr = nch * BITS, ngt = Ec / Q.group;
+    const int bit = lane * BITS, wi = bit >> 5, sh = bit & 31;
+    for (int u = warp; u < Er * nch; u += PW) {
+        const int tr = static_cast<int>(fdiv(static_cast<unsigned>(u), D.f_nchc)), ch = u - tr * nch;
+        const uint32_t *wsrc = S + tr * wpr + ch * BITS;
+        unsigned code = wsrc[wi] >> sh;
+        if (sh + BITS > 32) code |= wsrc[wi + 1] << (32 - sh);
+        T[tr * TCp + ch * 32 + lane] =
+            ssc[tr * ngt + static_cast<int>(fdiv(static_cast<unsigned>(ch), D.f_gch))] * lev[code & MASK];
     }
 }
 
-// Registers -> fp32 tile (forward sign factors applied when asked). The
-// codes input goes through the tail of each tile row: words first, then
-// every warp decodes its rows in place.
 template <int PRO>
-__device__ __forceinline__ void store_pre(const PassDesc &D, const QuantDev &Q, const Tabs &tb, float *T,
-                                          float *ssc, const float *lev, const Pre &R, bool signs, int tid,
-                                          int warp, int lane) {
+__device__ __forceinline__ void convert_input(const PassDesc &D, const QuantDev &Q, const Tabs &tb, const void *S,
+                                              float *T, const float *ssc, const float *lev, bool signs, int tid,
+                                              int warp, int lane) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     if constexpr (PRO == PRO_CODES) {
-        const int wpr = (Ec >> 5) * Q.bits, ngt = Ec / Q.group;
-#pragma unroll
-        for (int k = 0; k < NWR; ++k) {
-            const int i = tid + PT * k;
-            if (i < Er * wpr) {
-                const int tr = static_cast<int>(fdiv(static_cast<unsigned>(i), D.f_wpr)), w = i - tr * wpr;
-                reinterpret_cast<unsigned *>(T + tr * TCp + (Ec - wpr))[w] = R.w[k];
-            }
-        }
-        if (tid < Er * ngt) ssc[tid] = R.sc;
-        __syncthreads();
-        if (Q.bits == 2) decode_rows<2>(D, Q, T, ssc, lev, warp, lane);
-        else if (Q.bits == 3) decode_rows<3>(D, Q, T, ssc, lev, warp, lane);
-        else decode_rows<4>(D, Q, T, ssc, lev, warp, lane);
+        const uint32_t *W = static_cast<const uint32_t *>(S);
+        if (Q.bits == 2) decode_staged<2>(D, Q, W, T, ssc, lev, warp, lane);
+        else if (Q.bits == 3) decode_staged<3>(D, Q, W, T, ssc, lev, warp, lane);
+        else decode_staged<4>(D, Q, W, T, ssc, lev, warp, lane);
     } else {
         const int nch = (Ec + 31) >> 5, nu = ((Er + 3) >> 2) * nch;
-#pragma unroll
-        for (int k = 0; k < NQR; ++k) {
-            const int u = warp + PW * k;
+        for (int u = warp; u < nu; u += PW) {
             const Quad qd = quad_of(u, D.f_nch, Er, Ec, lane);
-            if (u < nu && qd.ok) {
-                float4 x;
-                if constexpr (PRO == PRO_F32) {
-                    x = make_float4(__uint_as_float(R.q[k].x), __uint_as_float(R.q[k].y),
-                                    __uint_as_float(R.q[k].z), __uint_as_float(R.q[k].w));
-                } else {
-                    x = make_float4(__uint_as_float(R.q[k].x << 16), __uint_as_float(R.q[k].x & 0xffff0000u),
-                                    __uint_as_float(R.q[k].y << 16), __uint_as_float(R.q[k].y & 0xffff0000u));
-                }
-                if (signs) {
-                    const float rs = tb.rsg[qd.tr];
-                    x.x *= rs * tb.csg[qd.tc];
-                    x.y *= rs * tb.csg[qd.tc + 1];
-                    x.z *= rs * tb.csg[qd.tc + 2];
-                    x.w *= rs * tb.csg[qd.tc + 3];
-                }
-                float *t = T + qd.tr * TCp + qd.tc;
-                t[0] = x.x;
-                t[1] = x.y;
-                t[2] = x.z;
-                t[3] = x.w;
+            if (!qd.ok) continue;
+            float4 x;
+            if constexpr (PRO == PRO_F32) {
+                x = *reinterpret_cast<const float4 *>(static_cast<const float *>(S) + qd.tr * Ec + qd.tc);
+            } else {
+                const uint2 t = *reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(S) +
+                                                                 qd.tr * Ec + qd.tc);
+                x = make_float4(__uint_as_float(t.x << 16), __uint_as_float(t.x & 0xffff0000u),
+                                __uint_as_float(t.y << 16), __uint_as_float(t.y & 0xffff0000u));
             }
+            if (signs) {
+                const float rs = tb.rsg[qd.tr];
+                x.x *= rs * tb.csg[qd.tc];
+                x.y *= rs * tb.csg[qd.tc + 1];
+                x.z *= rs * tb.csg[qd.tc + 2];
+                x.w *= rs * tb.csg[qd.tc + 3];
+            }
+            float *t = T + qd.tr * TCp + qd.tc;
+            t[0] = x.x;
+            t[1] = x.y;
+            t[2] = x.z;
+            t[3] = x.w;
         }
     }
 }
@@ -797,16 +767,19 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
     for (int i = tid; i < Ec; i += PT) cloc[i] = axis_global(D.ax[1], 0u, i);
     __syncthreads();
 
-    Pre R;
+    void *S = sm + D.stage_base;                        // staging buffer of the next tile's input
+    float sc_next;
     {
         const Buf B0 = buf_of(sm, D, 0);
         build_tables(D, B0, rloc, cloc, t, ld, tid);
         __syncthreads();
-        load_pre<PRO>(D, Q, B0.tb, R, tid, warp, lane);
+        sc_next = issue_input<PRO>(D, Q, B0.tb, S, tid);
         issue_coefs(D, B0.tb, B0.C, warp, lane);
         cp_async_commit();
-        store_pre<PRO>(D, Q, B0.tb, T, B0.ssc, lev, R, load_signs, tid, warp, lane);
         cp_async_wait_all();
+        if (PRO == PRO_CODES && tid < Er * (Ec / Q.group)) B0.ssc[tid] = sc_next;
+        __syncthreads();
+        convert_input<PRO>(D, Q, B0.tb, S, T, B0.ssc, lev, load_signs, tid, warp, lane);
         __syncthreads();
     }
 
@@ -818,7 +791,7 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
         if (more) {
             build_tables(D, Bn, rloc, cloc, tn, ld, tid);
             __syncthreads();
-            load_pre<PRO>(D, Q, Bn.tb, R, tid, warp, lane);
+            sc_next = issue_input<PRO>(D, Q, Bn.tb, S, tid);
             issue_coefs(D, Bn.tb, Bn.C, warp, lane);
             cp_async_commit();
         }
@@ -844,8 +817,10 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
         __syncthreads();
 
         if (more) {
-            store_pre<PRO>(D, Q, Bn.tb, T, Bn.ssc, lev, R, load_signs, tid, warp, lane);
             cp_async_wait_all();
+            if (PRO == PRO_CODES && tid < Er * (Ec / Q.group)) Bn.ssc[tid] = sc_next;
+            __syncthreads();
+            convert_input<PRO>(D, Q, Bn.tb, S, T, Bn.ssc, lev, load_signs, tid, warp, lane);
             __syncthreads();
         }
     }
@@ -930,7 +905,7 @@ int tcp_of(int Ec) { return (Ec % 2 == 0) ? Ec + 1 : Ec; }
 // computed, one for the next), the tile-local index tables, then 16
 // dequantised levels.
 struct SmemLayout {
-    int tile_floats, coef_floats, tab_base, buf_floats, loc_base, lev_base, total_floats;
+    int tile_floats, coef_floats, tab_base, buf_floats, stage_base, loc_base, lev_base, total_floats;
 };
 
 SmemLayout smem_layout(const PlanInput &in, int iL, int jL, int iR, int jR, int Er, int Ec) {
@@ -941,7 +916,8 @@ SmemLayout smem_layout(const PlanInput &in, int iL, int jL, int iR, int jR, int 
     int b = L.tab_base + 2 * Er + 2 * Er + Er + 3 * Ec + Er + Ec;   // rin, rout (int64), rtab, ctab, cin, cout, signs
     if (Ec % in.group == 0) b += Er * (Ec / in.group);            // scales of a codes tile
     L.buf_floats = (b + 3) & ~3;
-    L.loc_base = L.tile_floats + 2 * L.buf_floats;
+    L.stage_base = L.tile_floats + 2 * L.buf_floats;
+    L.loc_base = L.stage_base + Er * Ec;                  // staging: fp32 tile (the largest input form)
     L.lev_base = L.loc_base + ((Er + Ec + 3) & ~3);
     L.total_floats = L.lev_base + 32;
     return L;
@@ -969,11 +945,11 @@ Cand best_tile(const PlanInput &in, int iL, int jL, int iR, int jR, bool first, 
             if (run % 4 || Ec % 4) continue;                // 16-byte f32 / 8-byte bf16 quads
             if (first && run < user_run) continue;          // the pass that reads (writes) the user matrix
             if (last && (Ec % in.group || Ec % 32)) continue;
-            if (last && Ec > 32 * MAXCH) continue;          // codes decode holds a row's chunks in registers
+            if (last && Ec > 32 * MAXCH) continue;          // quantised tiles at most 256 columns wide
             if (smem_layout(in, iL, jL, iR, jR, static_cast<int>(Er), static_cast<int>(Ec)).total_floats * 4 >
                 SMEM_BUDGET)
                 continue;
-            if (Er * Ec > NQR * 4 * PT) continue;           // register prefetch holds a whole tile
+            if (Er * Ec > TILE_MAX) continue;
             int64_t nv = TILE_MAX;
             if (hasL) nv = std::min<int64_t>(nv, Ec);
             if (hasR) nv = std::min<int64_t>(nv, Er);
@@ -1160,6 +1136,9 @@ void build_desc(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inver
     D.buf_floats = L.buf_floats;
     D.lev_base = L.lev_base;
     D.loc_base = L.loc_base;
+    D.stage_base = L.stage_base;
+    D.f_nq = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / 4)));
+    D.f_nchc = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / 32)));
     D.f_nch = make_fdiv(static_cast<unsigned>((D.ax[1].E + 31) / 32));
     D.f_wpr = make_fdiv(static_cast<unsigned>(std::max(1, (D.ax[1].E / 32) * in.bits)));
     D.f_ngt = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / in.group)));
