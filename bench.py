@@ -140,6 +140,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------ multi-rank helpers
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (every rank replicates the same step; the job
+    is done when the last replica is)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def job_gbs(world, steps, total_ms):
+    """Whole-job algorithmic GB/s: every rank processes STEP_BYTES per step."""
+    return world * STEP_BYTES * steps / (total_ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------ GPU arm
 
 def run_gpu(args, rank, world, local_rank):
@@ -226,11 +244,8 @@ def run_gpu(args, rank, world, local_rank):
             for k in range(npass):
                 kt[f"fwd_p{k}_{bits}bit"].append(ef[k].elapsed_time(ef[k + 1]))
                 kt[f"inv_p{k}_{bits}bit"].append(ei[k].elapsed_time(ei[k + 1]))
-    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = t.item()
         torch.distributed.barrier()
 
     # ---- end to end through the public two-sided calls, host buffers
@@ -267,12 +282,8 @@ def run_gpu(args, rank, world, local_rank):
             b.record(stream)
             b.synchronize()
             e_ms.append(a.elapsed_time(b))
-        e_total = sum(e_ms)
-        if world > 1:
-            t = torch.tensor([e_total], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_total = t.item()
-        e2e = {"value": round(world * STEP_BYTES * args.steps / (e_total * 1e-3) / 1e9, 2),
+        e_total = max_over_ranks(sum(e_ms), world, dev)
+        e2e = {"value": round(job_gbs(world, args.steps, e_total), 2),
                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_total / args.steps, 4),
                "api": "harp_rotate_quantize + harp_dequantize_unrotate (two-sided), pinned host buffers",
@@ -483,7 +494,7 @@ def main():
     if rank == 0:
         peaks, peak_src = load_peaks()
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        value = world * STEP_BYTES * args.steps / (total_ms * 1e-3) / 1e9
+        value = job_gbs(world, args.steps, total_ms)
         ktab = kernel_table(kt, npass, pass_fma)
         # dominant kernel: largest total time in the step
         dom = max(ktab, key=lambda k: ktab[k]["us"])
