@@ -50,6 +50,11 @@ WORKLOAD = ("4096x4096 bf16 weight (Student-t nu=3 x0.02, 0.5% input channels x2
             "dequantize+unrotate for each bit width")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 
+# DRAM bytes (read + write) per pass launch of this step, from one ncu capture
+# of the current pass kernels (profiles/pass_kernel_c2_4096x4096_traffic.md);
+# writes still in L2 when a launch ends are counted by the next launch.
+MEASURED_TRAFFIC = {"fwd_p0_2bit": 51849216, "fwd_p1_2bit": 88366848, "fwd_p2_2bit": 68218624, "inv_p0_2bit": 17544448, "inv_p1_2bit": 88150016, "inv_p2_2bit": 70254592, "fwd_p0_4bit": 48630272, "fwd_p1_4bit": 87965184, "fwd_p2_4bit": 68028160, "inv_p0_4bit": 21670144, "inv_p1_4bit": 88139520, "inv_p2_4bit": 70288896}
+
 
 def fwd_bytes_per_elem(bits):
     return 2.0 + bits / 8.0 + 2.0 / GROUP
@@ -502,7 +507,8 @@ def main():
         peak_tf = fp32_peak_tflops(smhz)
         d = ktab[dom]
         roof = {"kernel": dom, "bound": "alu", "achieved": d["tflops"], "peak": round(peak_tf, 1),
-                "unit": "TFLOP/s", "frac": round(d["tflops"] / peak_tf, 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(d["tflops"] / peak_tf, 4),
+                "traffic": MEASURED_TRAFFIC.get(dom),
                 "peak_source": f"FFMA: 148 SM x 128 lanes x 2 flop x {smhz:.0f} MHz (max SM clock, {peak_src})",
                 "algorithmic": f"2 flop per block coefficient per element: FMA per element by forward pass {pass_fma}",
                 "own_bytes_hbm_frac": round(d["own_gbs"] / hbm, 4)}
