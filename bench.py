@@ -25,6 +25,7 @@ no exchange step); the time is the maximum over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import shutil
@@ -322,8 +323,17 @@ def run_workloads(steps, dev):
         return a.elapsed_time(b) / steps * 1e-3
 
     out = {}
-    for name in ("c1", "c3", "c4", "c5"):
-        w = synth.workload(name)
+    for name in ("c1", "c3", "c4", "c5", "rht"):
+        if name == "rht":
+            # the c2 weight with Hadamard-initialised processors on both sides
+            # (random signs, normalised Sylvester blocks: HARP's theta = 0 start)
+            w = synth.workload("c2")
+            w = dataclasses.replace(w, name="rht_4096x4096",
+                           right=synth.side_draws(2, RADIX, "hadamard", synth.S_SIGNS_R, synth.S_BLOCKS_R),
+                           left=synth.side_draws(2, RADIX, "hadamard", synth.S_SIGNS_L, synth.S_BLOCKS_L),
+                           quants=[synth.Quant("lloyd_max", 4, GROUP)])
+        else:
+            w = synth.workload(name)
         rows, cols = w.rows, w.cols
         if w.dtype == "bf16":
             x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).to(dev)

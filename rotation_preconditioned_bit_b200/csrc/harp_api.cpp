@@ -36,6 +36,21 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 int cuda_status(int err) { return err == 0 ? HARP_OK : HARP_ERR_CUDA; }
 
+// Whether all n_groups blocks equal the normalised Sylvester Hadamard
+// matrix exactly, entry (i, j) = (-1)^popcount(i & j) / sqrt(b) in fp32
+// (HARP section 2.2: theta = 0 gives back G_b; b a power of two, 2..64).
+bool all_sylvester(int b, int64_t n_groups, const float *B) {
+    if (b < 2 || (b & (b - 1)) != 0) return false;
+    const float v = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+    for (int64_t c = 0; c < n_groups; ++c)
+        for (int i = 0; i < b; ++i)
+            for (int j = 0; j < b; ++j) {
+                const float e = (__builtin_popcount(static_cast<unsigned>(i & j)) & 1) ? -v : v;
+                if (B[(c * b + i) * b + j] != e) return false;
+            }
+    return true;
+}
+
 // Padded block shape of the pass kernels (see StageDev).
 int pass_jpad(int b) { return (b + 3) & ~3; }
 int pass_kp(int b) { return b <= 8 ? 8 : (b + 15) & ~15; }
@@ -342,6 +357,7 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
         p->dev.st[t].kp = pass_kp(b);
         p->dev.st[t].pfwd = base + poff[t];
         p->dev.st[t].pinv = base + poff[t] + static_cast<size_t>(d / b) * pass_jpad(b) * pass_kp(b);
+        p->dev.st[t].had = all_sylvester(b, d / b, blocks[t]) ? 1 : 0;
     }
     *out = p;
     return HARP_OK;

@@ -29,6 +29,10 @@ struct StageDev {
     int kp;
     const float *pfwd;
     const float *pinv;
+    // 1 when every block of the stage is exactly the normalised Sylvester
+    // Hadamard matrix (fp32 entries +-1/sqrt(b), b a power of two): the pass
+    // kernels then apply the stage as a fast Walsh-Hadamard butterfly.
+    int had;
 };
 
 struct PlanDev {

@@ -99,6 +99,7 @@ struct PStage {
     int gstride;      // floats per slot
     int64_t s;        // global stride of the digit
     const float *coef;  // [d/b][jpad][kp]
+    int had;          // every block is the normalised Sylvester Hadamard: butterfly, no coefficients
 };
 
 struct PassDesc {
@@ -338,6 +339,52 @@ __device__ __forceinline__ void stage_run(float *T, const float *C, const PStage
             __syncthreads();
             if (active) unit_store<K>(T, S.b, kc * K, step, p, vok, gok, acc);
             __syncthreads();
+        }
+    }
+}
+
+// A stage whose blocks are all the normalised Sylvester Hadamard matrix H_b
+// (HARP section 2.2, theta = 0): each lane keeps the b inputs of its
+// vectors in registers and applies the fast Walsh-Hadamard butterfly, log2 b
+// rounds of (a + c, a - c) on pairs h apart, which computes
+// sum_j (-1)^popcount(k & j) x_j for every output k, then scales by the
+// block entry 1/sqrt(b). In place: every lane writes only the elements it read.
+template <int B>
+__device__ __forceinline__ void stage_fwht(float *T, const PStage &S, int A, int Bv, int NV, int warp, int lane) {
+    const int LV = S.LV, LG = 32 / LV;
+    const int lv = lane & (LV - 1), lg = lane / LV;
+    const int span = LV * VL;
+    const int nvc = (NV + span - 1) / span;
+    const int ngb = (S.G + LG - 1) / LG;
+    const int step = S.sig * A;
+    const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(B)));
+    for (int u = warp; u < ngb * nvc; u += PW) {
+        const int gb = u / nvc, vc = u - gb * nvc;
+        const int gi = gb * LG + lg;
+        const bool gok = gi < S.G;
+        const int g = gok ? gi : S.G - 1;
+        const int base = (g / S.sig) * (S.b * S.sig) + g % S.sig;
+#pragma unroll
+        for (int v = 0; v < VL; ++v) {
+            const int vi = vc * span + lv + LV * v;
+            const bool ok = gok && vi < NV;
+            float *xp = T + base * A + min(vi, NV - 1) * Bv;
+            float x[B];
+#pragma unroll
+            for (int j = 0; j < B; ++j) x[j] = xp[j * step];
+#pragma unroll
+            for (int h = 1; h < B; h <<= 1)
+#pragma unroll
+                for (int i = 0; i < B; ++i)
+                    if ((i & h) == 0) {
+                        const float a = x[i], c = x[i + h];
+                        x[i] = a + c;
+                        x[i + h] = a - c;
+                    }
+            if (ok) {
+#pragma unroll
+                for (int j = 0; j < B; ++j) xp[j * step] = x[j] * scale;
+            }
         }
     }
 }
@@ -616,6 +663,7 @@ __device__ __forceinline__ void build_tables(const PassDesc &D, const Buf &B, co
 __device__ __forceinline__ void issue_coefs(const PassDesc &D, const Tabs &tb, float *C, int warp, int lane) {
     for (int u = 0; u < D.nst; ++u) {
         const PStage &S = D.st[u];
+        if (S.had) continue;
         const int cpg = S.jpad * S.kp / 4;
         const int *tab = S.axis == 0 ? tb.rtab : tb.ctab;
         for (int gi = warp; gi < S.G; gi += PW) {
@@ -800,7 +848,15 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
             const PStage &S = D.st[u];
             const bool rows = (S.axis == 0);
             const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
-            if (S.kp == 8) stage_run<8, false>(T, B.C, S, A, Bv, NV, warp, lane);
+            if (S.had) {
+                switch (S.b) {
+                    case 2: stage_fwht<2>(T, S, A, Bv, NV, warp, lane); break;
+                    case 4: stage_fwht<4>(T, S, A, Bv, NV, warp, lane); break;
+                    case 8: stage_fwht<8>(T, S, A, Bv, NV, warp, lane); break;
+                    case 16: stage_fwht<16>(T, S, A, Bv, NV, warp, lane); break;
+                    default: stage_fwht<32>(T, S, A, Bv, NV, warp, lane); break;
+                }
+            } else if (S.kp == 8) stage_run<8, false>(T, B.C, S, A, Bv, NV, warp, lane);
             else if (S.kp == 16) stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
             else stage_rounds(T, B.C, S, A, Bv, NV, warp, lane);
             __syncthreads();
@@ -887,11 +943,13 @@ struct PlanInput {
     int bits;
 };
 
+bool stage_is_fwht(const StageDev &s) { return s.had && s.b <= 32; }
+
 int stage_coef_floats(const PlanDev *pl, int i, int j, int E) {
     int f = 0;
     for (int t = i; t < j; ++t) {
         const StageDev &s = pl->st[t];
-        f += (E / s.b) * (s.jpad * s.kp + GPAD);
+        if (!stage_is_fwht(s)) f += (E / s.b) * (s.jpad * s.kp + GPAD);
     }
     return f;
 }
@@ -1078,7 +1136,8 @@ void fill_stages(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inve
         S.gstride = sd.jpad * sd.kp + GPAD;
         S.s = sd.s;
         S.coef = inverse ? sd.pinv : sd.pfwd;
-        coef_floats += S.G * S.gstride;
+        S.had = stage_is_fwht(sd) ? 1 : 0;
+        if (!S.had) coef_floats += S.G * S.gstride;
     }
 }
 

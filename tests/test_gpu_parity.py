@@ -350,3 +350,30 @@ def test_pass_events_time_each_pass():
     times = [evs[k].elapsed_time(evs[k + 1]) for k in range(n)]
     assert all(t > 0 for t in times)
     assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
+
+
+def test_hadamard_two_sided_matches_oracle():
+    """Hadamard-initialised processors on both sides (HARP section 2.2,
+    theta = 0: random signs times normalised Sylvester blocks), which the
+    pass kernels apply as Walsh-Hadamard butterflies: the forward rotation +
+    4-bit Lloyd-Max, and the inverse of a random code stream, match the
+    oracle."""
+    left_s = synth.side_draws(21, (16, 8, 8), "hadamard", synth.S_SIGNS_L, synth.S_BLOCKS_L)
+    right_s = synth.side_draws(21, (16, 16, 8), "hadamard", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    rows, cols = 1024, 2048
+    W = synth.small_matrix(22, rows, cols, outlier_cols=4, scale=0.02)
+    Wb = synth.to_bf16_bits(W)
+    Pl, Pr = oracle.processor(left_s), oracle.processor(right_s)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(synth.bf16_bits_to_f64(Wb), Pl, Pr, "lloyd_max", 4, 128)
+    left, right = harp.Plan.from_side(left_s), harp.Plan.from_side(right_s)
+    cb = harp.Codebook("lloyd_max", 4, 128)
+    assert harp.harp_pass_count(left, right, cb) >= 2
+    xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, rot = harp.rotate_quantize(left, right, cb, xb, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, 4, 128)
+    raw, sc = synth.random_code_stream(23, rows, cols, 4, 128)
+    ref3 = oracle.dequantize_unrotate(oracle.unpack(4, raw, cols), sc, Pl, Pr, "lloyd_max", 4, 128)
+    out = harp.dequantize_unrotate(left, right, cb, torch.from_numpy(raw).cuda(),
+                                   torch.from_numpy(sc.view(np.int16)).cuda(), rows, cols, torch.float32)
+    assert rel_l2(out.cpu().numpy(), ref3) <= TOL_F32
