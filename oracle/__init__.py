@@ -51,6 +51,7 @@ _D = ctypes.POINTER(ctypes.c_double)
 _I32 = ctypes.POINTER(ctypes.c_int32)
 _I64 = ctypes.POINTER(ctypes.c_int64)
 _U8 = ctypes.POINTER(ctypes.c_uint8)
+_I8 = ctypes.POINTER(ctypes.c_int8)
 _U16 = ctypes.POINTER(ctypes.c_uint16)
 _INT = ctypes.c_int
 _L = ctypes.c_int64
@@ -67,6 +68,8 @@ def _set_types(L):
     L.orc_givens.argtypes = [ctypes.c_double, _D]
     L.orc_givens.restype = None
     L.orc_stage_blocks.argtypes = [_INT, _INT, _L, _D, _D, ctypes.c_double, _D]
+    L.orc_theta_quantize.argtypes = [_L, _D, _I8, ctypes.POINTER(ctypes.c_float)]
+    L.orc_theta_blocks.argtypes = [_INT, _L, _I8, ctypes.c_double, _D, _D]
     L.orc_lloyd_max.argtypes = [_INT, _D, ctypes.POINTER(ctypes.c_int)]
     L.orc_f16_bits.argtypes = [ctypes.c_double]
     L.orc_f16_bits.restype = ctypes.c_uint16
@@ -171,6 +174,31 @@ def stage_blocks(kind, b, n_groups, gauss=None, base=None, skew_scale=0.0):
     bs = None if base is None else np.ascontiguousarray(base, dtype=np.float64)
     _chk(lib().orc_stage_blocks(BLOCK_KINDS[kind], b, n_groups, _p(g, _D), _p(bs, _D),
                                 float(skew_scale), _p(out, _D)), "stage_blocks")
+    return out
+
+
+def theta_quantize(theta):
+    """int8 storage of one stage's parameters: (q int8, scale float32)."""
+    t = np.ascontiguousarray(theta, dtype=np.float64).ravel()
+    q = np.empty(t.size, dtype=np.int8)
+    s = ctypes.c_float(0.0)
+    _chk(lib().orc_theta_quantize(t.size, _p(t, _D), _p(q, _I8), ctypes.byref(s)), "theta_quantize")
+    return q.reshape(np.shape(theta)), np.float32(s.value)
+
+
+def theta_blocks(b, q, scale, G=None):
+    """Blocks [n_groups, b, b] of one stage from int8 q [n_groups, b(b-1)/2]
+    (b = 2: [n_groups, 1]) and the float scale; G the base mixer or None for
+    the normalised Sylvester matrix."""
+    P = max(b * (b - 1) // 2, 1) if b > 1 else 0
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    n = int(q.shape[0])
+    if q.size != n * P:
+        raise ValueError("oracle: theta_blocks wants [n_groups, b(b-1)/2] values")
+    out = np.empty((n, b, b), dtype=np.float64)
+    g = None if G is None else np.ascontiguousarray(G, dtype=np.float64)
+    _chk(lib().orc_theta_blocks(b, n, _p(q, _I8), float(np.float32(scale)), _p(g, _D),
+                                _p(out, _D)), "theta_blocks")
     return out
 
 

@@ -344,6 +344,84 @@ done:
     return st;
 }
 
+/* ------------------------------------------------------ int8-stored parameters */
+
+/* int8 storage of one stage's parameters [HARP 2.4 "deployment efficiency":
+ * the parameters may be kept in int8]. The pages give no scheme; the reading
+ * here is symmetric per-stage absmax: scale = max|theta| / 127 rounded to
+ * float, q = clamp(rint(theta / scale), -127, 127), theta^ = scale * q. An
+ * all-zero stage gets scale 0 and q = 0. */
+int orc_theta_quantize(int64_t n, const double *theta, int8_t *q, float *scale)
+{
+    double amax = 0.0;
+    for (int64_t i = 0; i < n; ++i)
+        if (fabs(theta[i]) > amax) amax = fabs(theta[i]);
+    if (!(amax < INFINITY)) return ORC_BAD;
+    float s = (float)(amax / 127.0);
+    *scale = s;
+    for (int64_t i = 0; i < n; ++i) {
+        double v = (s > 0.0f) ? rint(theta[i] / (double)s) : 0.0;
+        if (v > 127.0) v = 127.0;
+        if (v < -127.0) v = -127.0;
+        q[i] = (int8_t)v;
+    }
+    return ORC_OK;
+}
+
+/* Blocks of one stage from int8-stored parameters [HARP 2.2]:
+ * B_c = Q(theta_c) G_b. Group c holds P = b(b-1)/2 stored values, the strict
+ * upper triangle of its skew-symmetric generator in row-major order
+ * ((0,1), (0,2), ..., (0,b-1), (1,2), ...); theta = scale * q.
+ *   b = 2: Q is the Givens rotation by the one angle theta_c.
+ *   b > 2: A[i][j] = theta (i < j), -theta (i > j), 0 on the diagonal, and Q
+ *          is the Cayley map (I - A)^-1 (I + A).
+ *   b = 1: Q = [1].
+ * G: the base mixer [b][b] (float values promoted), or NULL for the
+ * normalised Sylvester matrix (b a power of two).
+ * out: [n_groups][b][b] row-major (out k, in j). */
+int orc_theta_blocks(int b, int64_t n_groups, const int8_t *q, double scale,
+                     const double *G, double *out)
+{
+    if (b < 1) return ORC_BAD;
+    const int64_t P = (int64_t)b * (b - 1) / 2;
+    double *Gm = (double *)malloc(sizeof(double) * b * b);
+    double *A = (double *)malloc(sizeof(double) * b * b);
+    double *Qm = (double *)malloc(sizeof(double) * b * b);
+    int st = ORC_OK;
+    if (!Gm || !A || !Qm) { st = ORC_BAD; goto done; }
+    if (G) memcpy(Gm, G, sizeof(double) * b * b);
+    else if ((st = orc_sylvester(b, Gm)) != ORC_OK) goto done;
+    for (int64_t c = 0; c < n_groups; ++c) {
+        const int8_t *qc = q + c * P;
+        if (b == 1) {
+            Qm[0] = 1.0;
+        } else if (b == 2) {
+            orc_givens(scale * (double)qc[0], Qm);
+        } else {
+            int64_t e = 0;
+            for (int i = 0; i < b; ++i) A[i * b + i] = 0.0;
+            for (int i = 0; i < b; ++i)
+                for (int j = i + 1; j < b; ++j, ++e) {
+                    A[i * b + j] = scale * (double)qc[e];
+                    A[j * b + i] = -A[i * b + j];
+                }
+            if ((st = orc_cayley(b, A, Qm)) != ORC_OK) goto done;
+        }
+        double *B = out + c * (int64_t)b * b;
+        for (int i = 0; i < b; ++i)
+            for (int j = 0; j < b; ++j) {
+                double acc = 0.0;
+                for (int k = 0; k < b; ++k) acc += Qm[i * b + k] * Gm[k * b + j];
+                B[i * b + j] = acc;
+            }
+    }
+done:
+    free(Gm);
+    free(A);
+    free(Qm);
+    return st;
+}
+
 /* ------------------------------------------------------------------ quantizer */
 
 /* Standard normal density and distribution function. */

@@ -253,6 +253,18 @@ def small_matrix(seed: int, rows: int, cols: int, outlier_cols: int = 0,
     return x
 
 
+S_THETA = 500       # + stage index: int8-stored stage parameters
+
+
+def theta_draws(seed: int, stage: int, n_groups: int, b: int, spread: float = 40.0):
+    """Stored int8 stage parameters: [n_groups, b(b-1)/2] values (one for
+    b = 2, none for b = 1), rint(spread * N(0,1)) clipped to [-127, 127], as a
+    trained stage kept in int8 would look."""
+    p = b * (b - 1) // 2 if b > 2 else (1 if b == 2 else 0)
+    g = normal(seed, S_THETA + stage, n_groups * p)
+    return np.clip(np.rint(spread * g), -127, 127).astype(np.int8).reshape(n_groups, p)
+
+
 def random_code_stream(seed: int, rows: int, cols: int, bits: int, group: int,
                        scale_lo: float = 0.01, scale_hi: float = 0.05):
     """Random inputs for the inverse path: packed code bytes (any byte string

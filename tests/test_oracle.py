@@ -139,6 +139,79 @@ def test_stage_blocks_kinds():
                                atol=1e-15)
 
 
+# ------------------------------------------------------------ int8-stored parameters
+
+def test_theta_quantize_reading():
+    theta = 0.05 * RNG.standard_normal(1000)
+    theta[17] = -0.4                                  # the stage's absmax
+    q, s = oracle.theta_quantize(theta)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert s == np.float32(0.4 / 127)
+    assert q[17] == -127 and np.abs(q).max() == 127
+    # round to nearest: every stored value within half a step of the original
+    assert np.all(np.abs(theta - np.float64(s) * q) <= 0.5 * np.float64(s) * (1 + 1e-12))
+    q0, s0 = oracle.theta_quantize(np.zeros(12))
+    assert s0 == 0 and not q0.any()
+
+
+def _skew_from_upper(b, vals):
+    """Skew-symmetric matrix whose strict upper triangle, read row by row, is
+    vals (numpy's triu_indices order)."""
+    A = np.zeros((b, b))
+    iu = np.triu_indices(b, 1)
+    A[iu] = vals
+    return A - A.T
+
+
+@pytest.mark.parametrize("b", [3, 4, 16, 32])
+def test_theta_blocks_cayley_against_library_solve(b):
+    n, P = 4, b * (b - 1) // 2
+    q = RNG.integers(-127, 128, size=(n, P)).astype(np.int8)
+    scale = np.float32(0.002)
+    if (b & (b - 1)) == 0:
+        G = sylvester_closed_form(b)
+        B = oracle.theta_blocks(b, q, scale)
+    else:
+        G = np.linalg.qr(RNG.standard_normal((b, b)))[0]
+        B = oracle.theta_blocks(b, q, scale, G)
+    for c in range(n):
+        A = _skew_from_upper(b, np.float64(scale) * q[c].astype(np.float64))
+        ref = np.linalg.solve(np.eye(b) - A, np.eye(b) + A) @ G
+        np.testing.assert_allclose(B[c], ref, atol=1e-13)
+        np.testing.assert_allclose(B[c].T @ B[c], np.eye(b), atol=1e-13)
+    # a single nonzero generator entry (0, 2): A = a(E02 - E20); the Cayley map
+    # of a plane rotation generator is the rotation by 2 atan(a) in that plane
+    qs = np.zeros((1, P), np.int8)
+    qs[0, 1] = 100
+    a = np.float64(scale) * 100
+    R = np.eye(b)
+    phi = 2 * math.atan(a)
+    R[0, 0] = R[2, 2] = math.cos(phi)
+    R[0, 2], R[2, 0] = math.sin(phi), -math.sin(phi)      # A[0][2] = +a
+    Gp = None if (b & (b - 1)) == 0 else G
+    np.testing.assert_allclose(oracle.theta_blocks(b, qs, scale, Gp)[0], R @ G, atol=1e-14)
+
+
+def test_theta_blocks_zero_givens_and_trivial():
+    # theta = 0 gives back the base mixer exactly (HARP 2.2 initialisation)
+    for b in (2, 8, 16, 64):
+        P = max(b * (b - 1) // 2, 1)
+        Z = oracle.theta_blocks(b, np.zeros((3, P), np.int8), np.float32(0.01))
+        np.testing.assert_array_equal(Z, np.broadcast_to(sylvester_closed_form(b), (3, b, b)))
+    # b = 2: Givens rotation by scale * q times H_2, closed form
+    q = np.array([[37], [-128], [0]], np.int8)
+    s = np.float32(0.01)
+    B = oracle.theta_blocks(2, q, s)
+    for c in range(3):
+        a = np.float64(s) * int(q[c, 0])
+        ca, sa = math.cos(a), math.sin(a)
+        ref = np.array([[ca - sa, ca + sa], [sa + ca, sa - ca]]) / math.sqrt(2)
+        np.testing.assert_allclose(B[c], ref, atol=1e-15)
+    # b = 1: every block is [1] (no parameters)
+    np.testing.assert_array_equal(oracle.theta_blocks(1, np.zeros((5, 0), np.int8), s),
+                                  np.ones((5, 1, 1)))
+
+
 # ------------------------------------------------------------ processor
 
 @pytest.mark.parametrize("radix", [(16, 16), (2, 4, 8), (4, 4, 4, 4), (256,), (2,) * 8])
