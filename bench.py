@@ -362,6 +362,42 @@ def run_workloads(steps, dev):
             out[key] = rec
         del x, ws
         torch.cuda.empty_cache()
+    out.update(run_theta_loads(timed, dev))
+    return out
+
+
+def run_theta_loads(timed, dev):
+    """Device time to rebuild every stage of a processor from int8-stored
+    parameters (harp_plan_load_theta: Givens / Cayley times the base mixer,
+    double precision), for the 4096x4096 and 8192x28672 processors."""
+    import numpy as np
+    import torch
+
+    import rotation_preconditioned_bit_b200 as harp
+    from rotation_preconditioned_bit_b200 import synth
+
+    out = {}
+    for name, radix in (("theta_4096_16x16x16", (16, 16, 16)), ("theta_28672_7x16x16x16", (7, 16, 16, 16)),
+                        ("theta_8192_32x16x16", (32, 16, 16))):
+        d = int(np.prod(radix))
+        side = synth.side_draws(5, radix, "hadamard", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+        plan = harp.Plan.from_side(side)
+        params = []
+        for t, b in enumerate(radix):
+            q = torch.from_numpy(synth.theta_draws(5, t, d // b, b)).to(dev)
+            base = None
+            if b & (b - 1):
+                base = torch.from_numpy(harp.stage_blocks("hadamard", b, 1, None, side.base[t])[0]).to(dev)
+            params.append((q, base))
+
+        def load():
+            for t, (q, base) in enumerate(params):
+                harp.harp_plan_load_theta(plan, t, q, 0.05 / 40, base)
+
+        t_load = timed(load)
+        groups = sum(d // b for b in radix)
+        out[name] = {"stages": len(radix), "groups": groups, "us": round(t_load * 1e6, 2),
+                     "blocks_per_s": float(f"{groups / t_load:.4g}")}
     return out
 
 

@@ -147,6 +147,44 @@ int harp_plan_info(harp_plan_t plan, int64_t *d, int *m, int32_t *radix);
 int harp_stage_blocks(int kind, int b, int64_t n_groups, const double *gauss,
                       const double *base_gauss, double skew_scale, float *out);
 
+/* Build one stage's blocks on the device from int8-stored parameters
+ * [HARP 2.2 (B = Q(theta) G_b; Givens for b = 2, Cayley for b > 2),
+ *  HARP 2.4 (parameters stored in int8)]:
+ *    B_c = Q(theta_c) G_b,  theta = theta_scale * q.
+ *  b = 2: Q = [[cos a, -sin a], [sin a, cos a]], a = theta_c (one value).
+ *  b > 2: Q = (I - A)^-1 (I + A), A skew-symmetric whose strict upper
+ *         triangle, read row by row ((0,1), (0,2), ..., (0,b-1), (1,2), ...),
+ *         is theta_c's b(b-1)/2 values.
+ *  b = 1: B = [1].
+ * Computed in double precision on the device, rounded once to float. Every q
+ * = 0 gives G_b exactly.
+ *  b            1..HARP_MAX_RADIX.
+ *  theta        device int8 [n_groups][P], P = b(b-1)/2 (1 for b = 2, 0 for
+ *               b = 1; may be NULL then).
+ *  theta_scale  the stage's scale (finite).
+ *  base         device float [b][b] row-major G_b, required when b is not a
+ *               power of two; NULL = the normalised Sylvester matrix
+ *               (-1)^popcount(k & j) / sqrt(b).
+ *  out          device float [n_groups][b][b] row-major (out k, in j),
+ *               4-byte aligned.
+ * Stream-ordered and asynchronous. Errors: INVALID_ARG (NULL pointer,
+ * non-finite scale, missing base), UNSUPPORTED (b outside [1, 64]),
+ * ALIGNMENT, CUDA. */
+int harp_theta_blocks(int b, int64_t n_groups, const int8_t *theta, float theta_scale,
+                      const float *base, float *out, void *stream);
+
+/* Replace stage `stage` of a plan with the blocks harp_theta_blocks builds
+ * from (theta, theta_scale, base), on the device and in the plan's own
+ * layouts (the plan's radix b = radix[stage], n_groups = d / b). Stream-
+ * ordered: launches on `stream` before this call use the old blocks, later
+ * ones the new; launches on other streams must be ordered by the caller. The
+ * stage is afterwards applied by general block arithmetic (never the
+ * Walsh-Hadamard butterfly), also when every q is 0.
+ * Errors: INVALID_ARG (NULL plan or pointer, stage outside [0, m), non-finite
+ * scale, missing base), CUDA. */
+int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float theta_scale,
+                         const float *base, void *stream);
+
 /* Lloyd-Max centroids for N(0,1) with 2^bits levels  [PolarQuant 2], computed
  * on the host (double precision, rounded to float): ascending, odd-symmetric.
  * out: host [2^bits]. bits in {2, 3, 4}. */

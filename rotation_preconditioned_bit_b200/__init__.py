@@ -40,6 +40,7 @@ EXPORTS = (
     "harp_workspace_size", "harp_rotate", "harp_quantize", "harp_dequantize",
     "harp_rotate_quantize", "harp_dequantize_unrotate", "harp_rotate_quantize_static",
     "harp_pass_count", "harp_pass_fma", "harp_set_pass_events",
+    "harp_theta_blocks", "harp_plan_load_theta",
 )
 
 
@@ -87,6 +88,8 @@ def lib():
         L.harp_pass_fma.argtypes = [_P, _P, _P, _INT, ctypes.POINTER(_INT)]
         L.harp_set_pass_events.argtypes = [_P, _INT]
         L.harp_rotate_quantize_static.argtypes = [_P, _P, _P, _P, _INT, _I64, _I64, _P, _P, _P, _P]
+        L.harp_theta_blocks.argtypes = [_INT, _I64, _P, ctypes.c_float, _P, _P, _P]
+        L.harp_plan_load_theta.argtypes = [_P, _INT, _P, ctypes.c_float, _P, _P]
         _lib = L
     return _lib
 
@@ -314,6 +317,45 @@ def harp_rotate_quantize_static(left, right, cb, x, codes, scales, rotated_out=N
                                              _ptr(scales), _ptr(rotated_out), _stream(stream)),
            "harp_rotate_quantize_static")
     return codes, scales
+
+
+def _check_theta(b, theta, n_groups, base):
+    import torch
+    p = b * (b - 1) // 2 if b > 2 else (1 if b == 2 else 0)
+    if theta is not None and (theta.dtype != torch.int8 or not theta.is_contiguous()
+                              or theta.numel() != n_groups * p):
+        raise ValueError(f"theta must be a contiguous int8 tensor of {n_groups} x {p} values")
+    if base is not None and (base.dtype != torch.float32 or not base.is_contiguous()
+                             or base.numel() != b * b):
+        raise ValueError("base must be a contiguous float32 [b, b] tensor")
+
+
+def harp_theta_blocks(b, theta, theta_scale, out, base=None, stream=None):
+    """Blocks [n_groups, b, b] (float32 device tensor `out`) of one stage from
+    int8-stored parameters `theta` [n_groups, b(b-1)/2] (device int8) and the
+    stage's float scale; `base` the float32 [b, b] base mixer on the device,
+    or None for the normalised Sylvester matrix."""
+    import torch
+    _require_cuda(theta, out, base)
+    _check_theta(b, theta, out.shape[0], base)
+    if out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape[1:]) != (b, b):
+        raise ValueError("out must be a contiguous float32 [n_groups, b, b] tensor")
+    n = out.shape[0]
+    _check(lib().harp_theta_blocks(int(b), n, _ptr(theta), float(theta_scale), _ptr(base),
+                                   _ptr(out), _stream(stream)), "harp_theta_blocks")
+    return out
+
+
+def harp_plan_load_theta(plan, stage, theta, theta_scale, base=None, stream=None):
+    """Replace stage `stage` of `plan` with blocks built on the device from
+    int8-stored parameters (see harp_theta_blocks)."""
+    _require_cuda(theta, base)
+    b = plan.radix[stage] if 0 <= stage < len(plan.radix) else 0
+    if b:
+        _check_theta(b, theta, plan.d // b, base)
+    _check(lib().harp_plan_load_theta(plan.handle, int(stage), _ptr(theta), float(theta_scale),
+                                      _ptr(base), _stream(stream)), "harp_plan_load_theta")
+    return plan
 
 
 def harp_dequantize_unrotate(left, right, cb, codes, scales, out, workspace=None, stream=None):

@@ -178,6 +178,17 @@ bool lloyd_max_half(int K, std::vector<double> &pos) {
     return true;
 }
 
+// Argument checks shared by the two theta entry points.
+int theta_args_ok(int b, int64_t n_groups, const int8_t *theta, float theta_scale,
+                  const float *base) {
+    if (b < 1 || b > HARP_MAX_RADIX) return HARP_ERR_UNSUPPORTED;
+    if (n_groups < 0 || !std::isfinite(theta_scale)) return HARP_ERR_INVALID_ARG;
+    if (b > 1 && n_groups > 0 && !theta) return HARP_ERR_INVALID_ARG;
+    if ((b & (b - 1)) != 0 && !base) return HARP_ERR_INVALID_ARG;
+    if (base && !aligned(base, sizeof(float))) return HARP_ERR_ALIGNMENT;
+    return HARP_OK;
+}
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -368,6 +379,38 @@ int harp_plan_destroy(harp_plan_t plan) {
     int st = HARP_OK;
     if (plan->mem && cudaFree(plan->mem) != cudaSuccess) { cudaGetLastError(); st = HARP_ERR_CUDA; }
     delete plan;
+    return st;
+}
+
+int harp_theta_blocks(int b, int64_t n_groups, const int8_t *theta, float theta_scale,
+                      const float *base, float *out, void *stream) {
+    int st = theta_args_ok(b, n_groups, theta, theta_scale, base);
+    if (st) return st;
+    if (n_groups > 0 && !out) return HARP_ERR_INVALID_ARG;
+    if (!aligned(out, sizeof(float))) return HARP_ERR_ALIGNMENT;
+    harp::ThetaOut o{};
+    o.plain = out;
+    return cuda_status(harp::launch_theta_blocks(b, n_groups, theta, theta_scale, base, o, stream));
+}
+
+int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float theta_scale,
+                         const float *base, void *stream) {
+    if (!plan || stage < 0 || stage >= plan->m) return HARP_ERR_INVALID_ARG;
+    harp::StageDev &sd = plan->dev.st[stage];
+    const int b = sd.b;
+    const int64_t ng = plan->d / b;
+    int st = theta_args_ok(b, ng, theta, theta_scale, base);
+    if (st) return st;
+    harp::ThetaOut o{};
+    o.fwd = const_cast<float *>(sd.fwd);
+    o.inv = const_cast<float *>(sd.inv);
+    o.kpad = sd.kpad;
+    o.pfwd = const_cast<float *>(sd.pfwd);
+    o.pinv = const_cast<float *>(sd.pinv);
+    o.jp = sd.jpad;
+    o.kp = sd.kp;
+    st = cuda_status(harp::launch_theta_blocks(b, ng, theta, theta_scale, base, o, stream));
+    if (st == HARP_OK) sd.had = 0;
     return st;
 }
 

@@ -102,6 +102,23 @@ int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q
 // after pass k (k + 1 < n). Per calling thread.
 void set_pass_events(void *const *events, int n);
 
+// Stage blocks from int8-stored parameters (harp_theta.cu): B_c = Q(theta_c)
+// G_b for n_groups groups, theta = scale * q, written to every non-null
+// layout of ThetaOut. Returns a cudaError_t value.
+struct ThetaOut {
+    float *plain;   // [c][k][j] = B[k][j]
+    float *fwd;     // [(c b + j) kpad + k] = B[k][j]
+    float *inv;     // [(c b + k) kpad + j] = B[k][j]
+    int kpad;
+    float *pfwd;    // [(c jp + j) kp + k] = B[k][j]
+    float *pinv;    // [(c jp + k) kp + j] = B[k][j]
+    int jp;
+    int kp;
+};
+size_t theta_smem_bytes(int b);
+int launch_theta_blocks(int b, int64_t n_groups, const int8_t *theta, double scale,
+                        const float *base, const ThetaOut &o, void *stream);
+
 // Vectors per CTA the whole-vector kernel uses for this plan and epilogue
 // (0 if a vector does not fit in shared memory).
 int vec_tile(const PlanDev &plan, int epi, int group);

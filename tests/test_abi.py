@@ -160,3 +160,26 @@ def test_compute_calls_reject_bad_arguments_before_launch():
     n = ctypes.c_size_t()
     assert L.harp_workspace_size(None, None, 10, 20, ctypes.byref(n)) == 0 and n.value == 0
     assert L.harp_workspace_size(ctypes.c_void_p(8), None, 10, 20, ctypes.byref(n)) == 0 and n.value == 1600
+
+
+def test_theta_calls_reject_bad_arguments_before_launch():
+    L = harp.lib()
+    fake = ctypes.c_void_p(4096)
+    # radix outside [1, 64]
+    assert L.harp_theta_blocks(65, 1, fake, 0.01, None, fake, None) == 3
+    assert L.harp_theta_blocks(0, 1, fake, 0.01, None, fake, None) == 3
+    # missing parameters, output or base mixer (b = 5 is not a power of two)
+    assert L.harp_theta_blocks(4, 1, None, 0.01, None, fake, None) == 1
+    assert L.harp_theta_blocks(4, 1, fake, 0.01, None, None, None) == 1
+    assert L.harp_theta_blocks(5, 1, fake, 0.01, None, fake, None) == 1
+    # non-finite scale, negative group count
+    assert L.harp_theta_blocks(4, 1, fake, float("nan"), None, fake, None) == 1
+    assert L.harp_theta_blocks(4, 1, fake, float("inf"), None, fake, None) == 1
+    assert L.harp_theta_blocks(4, -1, fake, 0.01, None, fake, None) == 1
+    # misaligned output or base
+    assert L.harp_theta_blocks(4, 1, fake, 0.01, None, ctypes.c_void_p(4098), None) == 4
+    assert L.harp_theta_blocks(5, 1, fake, 0.01, ctypes.c_void_p(4098), fake, None) == 4
+    # no groups: nothing to do, no launch
+    assert L.harp_theta_blocks(4, 0, None, 0.01, None, None, None) == 0
+    # NULL plan
+    assert L.harp_plan_load_theta(None, 0, fake, 0.01, None, None) == 1
