@@ -542,11 +542,11 @@ int orc_quantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
                  const double *X, uint8_t *codes, uint16_t *scales,
                  double *margin, double *scale_margin)
 {
-    if (bits < 2 || bits > 4 || group <= 0 || cols % group) return ORC_BAD;
+    if (bits < 2 || bits > 5 || group <= 0 || cols % group) return ORC_BAD;
     int K = 1 << bits;
     int qmax = (1 << (bits - 1)) - 1;
-    double c64[16];
-    float cent[16], thr[16];
+    double c64[32];
+    float cent[32], thr[32];
     if (kind == 0) {
         if (orc_lloyd_max(bits, c64, NULL)) return ORC_BAD;
         orc_tables(bits, c64, cent, thr);
@@ -618,9 +618,9 @@ int orc_quantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
 int orc_dequantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
                    const uint8_t *codes, const uint16_t *scales, double *X)
 {
-    if (bits < 2 || bits > 4 || group <= 0 || cols % group) return ORC_BAD;
-    double c64[16];
-    float cent[16], thr[16];
+    if (bits < 2 || bits > 5 || group <= 0 || cols % group) return ORC_BAD;
+    double c64[32];
+    float cent[32], thr[32];
     if (kind == 0) {
         if (orc_lloyd_max(bits, c64, NULL)) return ORC_BAD;
         orc_tables(bits, c64, cent, thr);

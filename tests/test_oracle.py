@@ -377,7 +377,7 @@ def _mse(c):
                               epsabs=1e-14, epsrel=1e-12)[0] for k in range(K))
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
 def test_lloyd_max_fixed_point_by_quadrature(bits):
     """PolarQuant 2: MSE-optimal centroids for N(0,1): every level is the
     conditional mean of its cell (checked by numerical integration, not the
@@ -427,7 +427,7 @@ def _brute_nearest(z, levels):
     return np.argmin(np.abs(z[..., None] - levels[None, :]), axis=-1)
 
 
-@pytest.mark.parametrize("bits,group", [(2, 64), (3, 128), (4, 128), (4, 32)])
+@pytest.mark.parametrize("bits,group", [(2, 64), (3, 128), (4, 128), (4, 32), (5, 128)])
 def test_lloyd_max_codes_are_nearest_centroid(bits, group):
     X = synth.small_matrix(11 + bits, 16, 512, outlier_cols=3, scale=0.02)
     codes, scales, margin, smargin = oracle.quantize("lloyd_max", bits, group, X)
@@ -444,7 +444,7 @@ def test_lloyd_max_codes_are_nearest_centroid(bits, group):
     np.testing.assert_array_equal(scales, rms.astype(np.float16).view(np.uint16))
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
 def test_absmax_codes(bits):
     X = synth.small_matrix(21 + bits, 8, 256, outlier_cols=2)
     group = 128
@@ -488,7 +488,7 @@ def test_lloyd_max_dequantize_is_scaled_centroid():
 
 # ------------------------------------------------------------ packing
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
 def test_pack_matches_bitstream_brute_force(bits):
     cols = 64
     codes = RNG.integers(0, 1 << bits, (5, cols)).astype(np.uint8)
