@@ -70,6 +70,7 @@ def _set_types(L):
     L.orc_stage_blocks.argtypes = [_INT, _INT, _L, _D, _D, ctypes.c_double, _D]
     L.orc_theta_quantize.argtypes = [_L, _D, _I8, ctypes.POINTER(ctypes.c_float)]
     L.orc_theta_blocks.argtypes = [_INT, _L, _I8, ctypes.c_double, _D, _D]
+    L.orc_round_mid.argtypes = [_INT, _L, _D, _D]
     L.orc_lloyd_max.argtypes = [_INT, _D, ctypes.POINTER(ctypes.c_int)]
     L.orc_f16_bits.argtypes = [ctypes.c_double]
     L.orc_f16_bits.restype = ctypes.c_uint16
@@ -301,6 +302,29 @@ def rotate_quantize(X, left, right, kind, bits, group):
     Y = right.rotate_rows(Y)
     codes, scales, margin, smargin = quantize(kind, bits, group, Y)
     return Y, codes, pack(bits, codes), scales, margin, smargin
+
+
+MID_KINDS = {"f32": 0, "bf16": 1, "f16": 2}
+
+
+def round_mid(kind, X):
+    """X rounded (nearest even) to the storage type `kind` ('f32' | 'bf16' |
+    'f16', fp16 saturating at 65504), as float64."""
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    out = np.empty_like(X)
+    _chk(lib().orc_round_mid(MID_KINDS[kind], X.size, _p(X, _D), _p(out, _D)), "round_mid")
+    return out
+
+
+def requantize(codes, scales, right, kind_in, bits_in, group_in, mid, kind_out, bits_out, group_out):
+    """PolarQuant's two-stage codec [PQ 2-3]: dequantise the first-stage codes,
+    rotate the rows back, store the restored weights as `mid`, then quantise
+    them (no rotation) with the second quantiser.
+    Returns (restored, codes, packed, scales, margin, scale_margin)."""
+    Y = round_mid(mid, right.rotate_rows(dequantize(kind_in, bits_in, group_in, codes, scales),
+                                         inverse=True))
+    c2, s2, margin, smargin = quantize(kind_out, bits_out, group_out, Y)
+    return Y, c2, pack(bits_out, c2), s2, margin, smargin
 
 
 def dequantize_unrotate(codes, scales, left, right, kind, bits, group):

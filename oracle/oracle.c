@@ -613,6 +613,32 @@ int orc_quantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
     return ORC_OK;
 }
 
+/* Restored weights in a 16- or 32-bit storage type [PQ 3: the Q5 weights,
+ * dequantised and rotated back, are kept in fp16 and then handed to a
+ * downstream INT4 absmax quantiser]. Each value is rounded to nearest even
+ * from float64: kind 0 float, 1 bfloat16 (normal range), 2 fp16 (saturating
+ * at +-65504, the same conversion as the scales). */
+int orc_round_mid(int kind, int64_t n, const double *x, double *out)
+{
+    if (kind < 0 || kind > 2) return ORC_BAD;
+    for (int64_t i = 0; i < n; ++i) {
+        double v = x[i], a = fabs(v), r;
+        if (kind == 0) {
+            r = (double)(float)a;
+        } else if (kind == 2) {
+            r = orc_f16_value(orc_f16_bits(a));
+        } else if (a == 0.0) {
+            r = 0.0;
+        } else {
+            int e;
+            (void)frexp(a, &e);                     /* a = f 2^e, f in [0.5, 1) */
+            r = ldexp(nearbyint(ldexp(a, 8 - e)), e - 8);   /* 8 significant bits */
+        }
+        out[i] = (v < 0.0) ? -r : r;
+    }
+    return ORC_OK;
+}
+
 /* Dequantise: x = s * c[code] (Lloyd-Max, fp32 centroid table) or
  * x = s * (code - 2^(b-1)) (absmax). */
 int orc_dequantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,

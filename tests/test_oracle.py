@@ -540,3 +540,46 @@ def test_rotation_gaussianises_heavy_tails():
     kx = np.mean(x ** 4) / np.mean(x ** 2) ** 2
     ky = np.mean(y ** 4) / np.mean(y ** 2) ** 2
     assert kx > 6 and abs(ky - 3.0) < 0.5
+
+
+# ------------------------------------------------------------ two-stage codec
+
+def test_round_mid_against_library_casts():
+    import torch
+    x = np.concatenate([RNG.standard_normal(4000) * 10.0 ** RNG.integers(-6, 4, 4000),
+                        [0.0, -0.0, 65504.0, -65504.0]]).astype(np.float32).astype(np.float64)
+    f16 = oracle.round_mid("f16", x)
+    np.testing.assert_array_equal(f16, x.astype(np.float16).astype(np.float64))
+    # saturation past the largest fp16 (the reading used for the scales too)
+    np.testing.assert_array_equal(oracle.round_mid("f16", np.array([1e6, -70000.0])), [65504.0, -65504.0])
+    # bf16 from float32-representable values: one rounding, as torch's cast
+    bf = oracle.round_mid("bf16", x)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(bf, ref)
+    # exact ties go to the even neighbour (8 significant bits)
+    ties = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 3 * 2.0 ** -9 * 2.0 ** -7])
+    np.testing.assert_array_equal(oracle.round_mid("bf16", ties)[:3], [1.0, 1 + 2.0 ** -6, -1.0])
+    np.testing.assert_array_equal(oracle.round_mid("f32", x[:10] + 1e-12),
+                                  (x[:10] + 1e-12).astype(np.float32).astype(np.float64))
+
+
+def test_requantize_order_of_steps():
+    """PolarQuant sections 2-3: first-stage codes are dequantised, rotated
+    back (rows: r -> M^T r, i.e. X -> X M with the dense processor matrix),
+    stored as fp16, then quantised by the second quantiser without rotation."""
+    P = random_processor((8, 4, 4), RNG)
+    d = P.d
+    rows = 6
+    X = synth.small_matrix(3, rows, d, outlier_cols=2)
+    codes, scales, _, _ = oracle.quantize("lloyd_max", 5, 128, P.rotate_rows(X))
+    Y, c2, packed, s2, margin, _ = oracle.requantize(codes, scales, P, "lloyd_max", 5, 128,
+                                                     "f16", "absmax", 4, 64)
+    Xh = oracle.dequantize("lloyd_max", 5, 128, codes, scales)
+    np.testing.assert_allclose(Y, (Xh @ P.dense()).astype(np.float16), rtol=1e-3, atol=1e-6)
+    np.testing.assert_array_equal(Y, Y.astype(np.float16).astype(np.float64))
+    # the second stage is plain absmax on the restored fp16 weights
+    s = np.repeat(np.array([[oracle.f16_value(v) for v in r] for r in s2]), 64, axis=1)
+    Yg = np.abs(Y).reshape(rows, -1, 64).max(axis=2)
+    np.testing.assert_allclose(s[:, ::64], Yg / 7, rtol=1e-3)
+    assert np.all(np.abs(Y - s * (c2.astype(int) - 8)) <= 0.5 * s * (1 + 1e-2))
+    np.testing.assert_array_equal(packed, oracle.pack(4, c2))
