@@ -362,8 +362,40 @@ def run_workloads(steps, dev):
             out[key] = rec
         del x, ws
         torch.cuda.empty_cache()
+    out.update(run_polarquant(timed, dev))
     out.update(run_theta_loads(timed, dev))
     return out
+
+
+def run_polarquant(timed, dev):
+    """PolarQuant's per-block workload on the 4096x4096 bf16 weight: rows of
+    128 rotated by H_128 (radices (16, 8), Sylvester blocks, no signs) with
+    5-bit Lloyd-Max codes (Q5), its inverse, and the fused two-stage codec
+    (Q5 codes -> restored fp16 weights -> 4-bit absmax g128)."""
+    import numpy as np
+    import torch
+
+    import rotation_preconditioned_bit_b200 as harp
+    from rotation_preconditioned_bit_b200 import synth
+
+    rows = cols = 4096
+    n = rows * cols // 128
+    w = synth.workload("c2")
+    x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).to(dev).view(n, 128)
+    plan = harp.Plan((16, 8), [harp.stage_blocks("hadamard", b, 128 // b) for b in (16, 8)])
+    q5, a4 = harp.Codebook("lloyd_max", 5, 128), harp.Codebook("absmax", 4, 128)
+    c5, s5 = harp.empty_codes(n, 128, q5, dev)
+    c4, s4 = harp.empty_codes(n, 128, a4, dev)
+    o = torch.empty((n, 128), dtype=torch.bfloat16, device=dev)
+    e = rows * cols
+    t_f = timed(lambda: harp.harp_rotate_quantize(None, plan, q5, x, c5, s5))
+    t_i = timed(lambda: harp.harp_dequantize_unrotate(None, plan, q5, c5, s5, o))
+    t_r = timed(lambda: harp.harp_requantize(plan, q5, c5, s5, n, 128, "f16", a4, c4, s4))
+    b5, b4 = 5 / 8 + 2 / 128, 4 / 8 + 2 / 128
+    return {"polarquant_h128_q5_4096x4096": {
+        "fwd_us": round(t_f * 1e6, 2), "fwd_gbs": round(e * (2 + b5) / t_f / 1e9, 2),
+        "inv_us": round(t_i * 1e6, 2), "inv_gbs": round(e * (b5 + 2) / t_i / 1e9, 2),
+        "requant_q5_to_int4_us": round(t_r * 1e6, 2), "requant_gbs": round(e * (b5 + b4) / t_r / 1e9, 2)}}
 
 
 def run_theta_loads(timed, dev):

@@ -72,14 +72,14 @@ typedef enum harp_status {
     HARP_OK = 0,
     HARP_ERR_INVALID_ARG = 1,   /* NULL where a pointer is required, bad enum value */
     HARP_ERR_SHAPE = 2,         /* prod b_t != d, d != rows/cols, group does not divide cols, ... */
-    HARP_ERR_UNSUPPORTED = 3,   /* radix outside [1, 64], more than 16 stages, bits not in {2,3,4} */
+    HARP_ERR_UNSUPPORTED = 3,   /* radix outside [1, 64], more than 16 stages, bits not in {2,3,4,5} */
     HARP_ERR_ALIGNMENT = 4,     /* device pointer or leading dimension not aligned (see each call) */
     HARP_ERR_WORKSPACE = 5,     /* workspace NULL or smaller than harp_workspace_size() */
     HARP_ERR_CUDA = 6,          /* CUDA runtime error (no device, launch failure) */
     HARP_ERR_ALLOC = 7          /* host or device allocation failed at plan / codebook creation */
 } harp_status;
 
-enum harp_dtype { HARP_F32 = 0, HARP_BF16 = 1 };
+enum harp_dtype { HARP_F32 = 0, HARP_BF16 = 1, HARP_F16 = 2 /* harp_requantize's restored weights only */ };
 enum harp_side { HARP_RIGHT = 0, HARP_LEFT = 1 };
 enum harp_dir { HARP_FWD = 0, HARP_INV = 1 };
 enum harp_quant_kind { HARP_LLOYD_MAX = 0, HARP_ABSMAX = 1 };
@@ -187,12 +187,12 @@ int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float
 
 /* Lloyd-Max centroids for N(0,1) with 2^bits levels  [PolarQuant 2], computed
  * on the host (double precision, rounded to float): ascending, odd-symmetric.
- * out: host [2^bits]. bits in {2, 3, 4}. */
+ * out: host [2^bits]. bits in {2, 3, 4, 5} (5 = PolarQuant's Q5). */
 int harp_lloyd_max_centroids(int bits, float *out);
 
 /* Create a quantizer description  [PolarQuant 1, 2].
  *  kind       HARP_LLOYD_MAX or HARP_ABSMAX.
- *  bits       2, 3 or 4.
+ *  bits       2, 3, 4 or 5 (PolarQuant section 3 uses 5-bit Q5 codes).
  *  group      elements per scale group along a row: a positive multiple of
  *             32 (UNSUPPORTED otherwise); must divide cols at each call
  *             (group = cols gives one scale per row).
@@ -259,6 +259,32 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
                          const void *in, int in_dtype, int64_t rows, int64_t cols,
                          uint8_t *codes, uint16_t *scales, float *rotated_out,
                          void *workspace, size_t ws_bytes, void *stream);
+
+/* PolarQuant's two-stage codec, fused [PolarQuant 2 (codes, fp16 norm,
+ * H^-1 = H), 3 (Q5 weights restored to FP16, then a downstream absmax INT4
+ * quantizer)]: for every row,
+ *     restored = round_mid( D_s B_0^T ... B_{m-1}^T dequant_in(codes_in) )
+ *     (codes_out, scales_out) = quantize_out(restored)     (no rotation)
+ * i.e. harp_dequantize_unrotate (right side only) into the storage type
+ * `mid_dtype`, then harp_quantize with `cb_out`, in one pass over the matrix.
+ *  right        the first stage's row processor; right->d == cols.
+ *  cb_in        the first stage's codebook (any kind, 2..5 bits).
+ *  codes_in, scales_in  device, laid out as harp_quantize writes them.
+ *  mid_dtype    HARP_F32, HARP_BF16 or HARP_F16: each restored value is
+ *               rounded to nearest even in this type (fp16 saturating at
+ *               +-65504) before the second quantizer sees it.
+ *  restored_out optional device [rows x cols] contiguous array of
+ *               `mid_dtype` receiving the restored weights (NULL = none).
+ *  cb_out       the second codebook (e.g. HARP_ABSMAX, 4 bits, group 128).
+ *  codes_out, scales_out  device, as harp_quantize writes them for cb_out.
+ * Both groups must divide cols. Alignment: codes 4 bytes, scales 2 bytes,
+ * restored_out 16 bytes. Errors: INVALID_ARG, SHAPE, UNSUPPORTED (a row of
+ * `cols` values does not fit the kernel's shared-memory tile), ALIGNMENT,
+ * CUDA. */
+int harp_requantize(harp_plan_t right, harp_codebook_t cb_in, const uint8_t *codes_in,
+                    const uint16_t *scales_in, int64_t rows, int64_t cols, int mid_dtype,
+                    void *restored_out, harp_codebook_t cb_out, uint8_t *codes_out,
+                    uint16_t *scales_out, void *stream);
 
 /* Fused inverse path: dequantize, then W = M_L^T W' M_R  [HARP 5;
  * PolarQuant 2]. out: device [rows x cols] contiguous, F32 or BF16.

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libharp.so")
 
 HARP_OK = 0
-HARP_F32, HARP_BF16 = 0, 1
+HARP_F32, HARP_BF16, HARP_F16 = 0, 1, 2
 HARP_RIGHT, HARP_LEFT = 0, 1
 HARP_FWD, HARP_INV = 0, 1
 HARP_LLOYD_MAX, HARP_ABSMAX = 0, 1
@@ -40,7 +40,7 @@ EXPORTS = (
     "harp_workspace_size", "harp_rotate", "harp_quantize", "harp_dequantize",
     "harp_rotate_quantize", "harp_dequantize_unrotate", "harp_rotate_quantize_static",
     "harp_pass_count", "harp_pass_fma", "harp_set_pass_events",
-    "harp_theta_blocks", "harp_plan_load_theta",
+    "harp_theta_blocks", "harp_plan_load_theta", "harp_requantize",
 )
 
 
@@ -90,6 +90,7 @@ def lib():
         L.harp_rotate_quantize_static.argtypes = [_P, _P, _P, _P, _INT, _I64, _I64, _P, _P, _P, _P]
         L.harp_theta_blocks.argtypes = [_INT, _I64, _P, ctypes.c_float, _P, _P, _P]
         L.harp_plan_load_theta.argtypes = [_P, _INT, _P, ctypes.c_float, _P, _P]
+        L.harp_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _INT, _P, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -356,6 +357,21 @@ def harp_plan_load_theta(plan, stage, theta, theta_scale, base=None, stream=None
     _check(lib().harp_plan_load_theta(plan.handle, int(stage), _ptr(theta), float(theta_scale),
                                       _ptr(base), _stream(stream)), "harp_plan_load_theta")
     return plan
+
+
+_MID_CODES = {"f32": 0, "bf16": 1, "f16": 2}
+
+
+def harp_requantize(right, cb_in, codes_in, scales_in, rows, cols, mid, cb_out, codes_out,
+                    scales_out, restored_out=None, stream=None):
+    """PolarQuant's two-stage codec in one pass: dequantise `codes_in` with
+    cb_in, rotate the rows back with `right`, round to `mid` ('f32' | 'bf16'
+    | 'f16'; optionally stored in `restored_out`), quantise with cb_out."""
+    _require_cuda(codes_in, scales_in, codes_out, scales_out, restored_out)
+    _check(lib().harp_requantize(right.handle, cb_in.handle, _ptr(codes_in), _ptr(scales_in), rows, cols,
+                                 _MID_CODES[mid], _ptr(restored_out), cb_out.handle, _ptr(codes_out),
+                                 _ptr(scales_out), _stream(stream)), "harp_requantize")
+    return codes_out, scales_out
 
 
 def harp_dequantize_unrotate(left, right, cb, codes, scales, out, workspace=None, stream=None):

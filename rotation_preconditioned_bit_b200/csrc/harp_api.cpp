@@ -262,7 +262,7 @@ int harp_stage_blocks(int kind, int b, int64_t n_groups, const double *gauss,
 
 int harp_lloyd_max_centroids(int bits, float *out) {
     if (!out) return HARP_ERR_INVALID_ARG;
-    if (bits < 2 || bits > 4) return HARP_ERR_UNSUPPORTED;
+    if (bits < 2 || bits > 5) return HARP_ERR_UNSUPPORTED;
     const int K = 1 << bits;
     std::vector<double> pos;
     lloyd_max_half(K, pos);
@@ -427,7 +427,7 @@ int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group
     if (!out) return HARP_ERR_INVALID_ARG;
     *out = nullptr;
     if (kind != HARP_LLOYD_MAX && kind != HARP_ABSMAX) return HARP_ERR_INVALID_ARG;
-    if (bits < 2 || bits > 4) return HARP_ERR_UNSUPPORTED;
+    if (bits < 2 || bits > 5) return HARP_ERR_UNSUPPORTED;
     if (group <= 0) return HARP_ERR_SHAPE;
     if (group % 32 != 0 || group > std::numeric_limits<int32_t>::max()) return HARP_ERR_UNSUPPORTED;
     harp_codebook_s *cb = new (std::nothrow) harp_codebook_s();
@@ -438,7 +438,7 @@ int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group
     cb->q.bits = bits;
     cb->q.group = static_cast<int>(group);
     if (kind == HARP_LLOYD_MAX) {
-        float c[16];
+        float c[32];
         if (centroids) {
             for (int k = 0; k < K; ++k) c[k] = centroids[k];
             for (int k = 0; k + 1 < K; ++k)
@@ -541,6 +541,13 @@ int harp_dequantize(harp_codebook_t cb, const uint8_t *codes, const uint16_t *sc
     return cuda_status(harp::launch_dequantize(cb->q, codes, scales, rows, cols, out, out_dtype, ld_out, stream));
 }
 
+// Whether a two-sided call runs as pass kernels (their quantizer epilogue and
+// code decoding handle 2- to 4-bit codes; 5-bit codes take the whole-vector
+// kernels).
+static bool use_passes(harp_plan_t left, harp_plan_t right, harp_codebook_t cb) {
+    return left && cb->q.bits <= 4 && harp::pass_plan_ok(left->dev, right->dev, cb->q.group);
+}
+
 static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int64_t rows,
                       int64_t cols, void *workspace, size_t ws_bytes) {
     if (!right || !cb) return HARP_ERR_INVALID_ARG;
@@ -548,7 +555,7 @@ static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, i
     if (st) return st;
     if (right->d != cols) return HARP_ERR_SHAPE;
     if (left && left->d != rows) return HARP_ERR_SHAPE;
-    if (!(left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group)) &&
+    if (!use_passes(left, right, cb) &&
         harp::vec_tile(right->dev, harp::EPI_QUANT, cb->q.group) == 0)
         return HARP_ERR_UNSUPPORTED;
     if (left) {
@@ -571,7 +578,7 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
     if (!aligned(in, 16) || !aligned(codes, 4) || !aligned(scales, 2) ||
         (rotated_out && !aligned(rotated_out, 16)) || cols % 4)
         return HARP_ERR_ALIGNMENT;
-    if (left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group))
+    if (use_passes(left, right, cb))
         return cuda_status(harp::launch_pass_fwd(left->dev, right->dev, cb->q, in, in_dtype, codes, scales,
                                                  rotated_out, static_cast<float *>(workspace), stream));
     const int pro_in = (in_dtype == HARP_F32) ? harp::PRO_F32 : harp::PRO_BF16;
@@ -608,9 +615,43 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
     return cuda_status(harp::launch_vec(right->dev, &cb->q, Lr, stream));
 }
 
+int harp_requantize(harp_plan_t right, harp_codebook_t cb_in, const uint8_t *codes_in,
+                    const uint16_t *scales_in, int64_t rows, int64_t cols, int mid_dtype,
+                    void *restored_out, harp_codebook_t cb_out, uint8_t *codes_out,
+                    uint16_t *scales_out, void *stream) {
+    if (!right || !cb_in || !cb_out) return HARP_ERR_INVALID_ARG;
+    if (mid_dtype != HARP_F32 && mid_dtype != HARP_BF16 && mid_dtype != HARP_F16) return HARP_ERR_INVALID_ARG;
+    int st = check_codec(cb_in, rows, cols);
+    if (st == HARP_OK) st = check_codec(cb_out, rows, cols);
+    if (st) return st;
+    if (right->d != cols) return HARP_ERR_SHAPE;
+    if (harp::vec_tile(right->dev, harp::EPI_REQUANT, cb_out->q.group, harp::PRO_CODES) == 0)
+        return HARP_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!codes_in || !scales_in || !codes_out || !scales_out) return HARP_ERR_INVALID_ARG;
+    if (!aligned(codes_in, 4) || !aligned(scales_in, 2) || !aligned(codes_out, 4) ||
+        !aligned(scales_out, 2) || (restored_out && !aligned(restored_out, 16)))
+        return HARP_ERR_ALIGNMENT;
+    harp::VecLaunch L{};
+    L.side = HARP_RIGHT;
+    L.dir = HARP_INV;
+    L.pro = harp::PRO_CODES;
+    L.epi = harp::EPI_REQUANT;
+    L.nvec = rows;
+    L.in_codes = codes_in;
+    L.in_scales = scales_in;
+    L.out = restored_out;
+    L.ld_out = cols;
+    L.codes = codes_out;
+    L.scales = scales_out;
+    L.q2 = cb_out->q;
+    L.mid = mid_dtype;
+    return cuda_status(harp::launch_vec(right->dev, &cb_in->q, L, stream));
+}
+
 int harp_pass_count(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int *passes) {
     if (!right || !cb || !passes) return HARP_ERR_INVALID_ARG;
-    *passes = (left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group)) ? harp::pass_count(left->dev, right->dev, cb->q.group) : 0;
+    *passes = use_passes(left, right, cb) ? harp::pass_count(left->dev, right->dev, cb->q.group) : 0;
     return HARP_OK;
 }
 
@@ -638,7 +679,7 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
     if (rows == 0 || cols == 0) return HARP_OK;
     if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
     if (!aligned(out, 16) || !aligned(scales, 2) || cols % 4) return HARP_ERR_ALIGNMENT;
-    if (left && harp::pass_plan_ok(left->dev, right->dev, cb->q.group))
+    if (use_passes(left, right, cb))
         return cuda_status(harp::launch_pass_inv(left->dev, right->dev, cb->q, codes, scales, out, out_dtype,
                                                  static_cast<float *>(workspace), stream));
     harp::VecLaunch Lr{};

@@ -47,12 +47,12 @@ struct QuantDev {
     int kind;       // HARP_LLOYD_MAX | HARP_ABSMAX
     int bits;
     int group;
-    float level[16];  // dequantised level per code (centroid or code - 2^(b-1))
-    float thr[16];    // Lloyd-Max midpoints (K - 1 used)
+    float level[32];  // dequantised level per code (centroid or code - 2^(b-1))
+    float thr[32];    // Lloyd-Max midpoints (K - 1 used)
 };
 
 enum Prologue { PRO_F32 = 0, PRO_BF16 = 1, PRO_CODES = 2 };
-enum Epilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_QUANT = 2, EPI_QUANT_F32 = 3 };
+enum Epilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_QUANT = 2, EPI_QUANT_F32 = 3, EPI_REQUANT = 4 };
 
 // Launch parameters of the whole-vector kernel: `nvec` vectors of length
 // plan.d taken from a row-major matrix, either its rows (side RIGHT) or its
@@ -71,6 +71,11 @@ struct VecLaunch {
     uint16_t *scales;      // EPI_QUANT*: [nvec][d/group]
     const uint8_t *in_codes;     // PRO_CODES
     const uint16_t *in_scales;   // PRO_CODES
+    // EPI_REQUANT: the second quantizer (codes / scales above are its
+    // outputs) and the restored weights' storage type (HARP_F32 | HARP_BF16 |
+    // HARP_F16); `out` (optional) receives the restored weights in that type.
+    QuantDev q2;
+    int mid;
 };
 
 // Returns a cudaError_t value (0 = success).
@@ -121,6 +126,6 @@ int launch_theta_blocks(int b, int64_t n_groups, const int8_t *theta, double sca
 
 // Vectors per CTA the whole-vector kernel uses for this plan and epilogue
 // (0 if a vector does not fit in shared memory).
-int vec_tile(const PlanDev &plan, int epi, int group);
+int vec_tile(const PlanDev &plan, int epi, int group, int pro = PRO_F32);
 
 }  // namespace harp

@@ -72,6 +72,21 @@ __device__ __forceinline__ unsigned short float_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// A value rounded (nearest even) to the restored weights' storage type:
+// float, bfloat16, or fp16 saturating at +-65504.
+__device__ __forceinline__ float round_mid(float v, int mid) {
+    if (mid == HARP_BF16) return bf16_bits_to_float(float_to_bf16_bits(v));
+    if (mid == HARP_F16) return __half2float(__float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f)));
+    return v;
+}
+
+// Store a value already rounded by round_mid (the conversion is exact).
+__device__ __forceinline__ void store_mid(void *base, int64_t off, float v, int mid) {
+    if (mid == HARP_BF16) static_cast<unsigned short *>(base)[off] = float_to_bf16_bits(v);
+    else if (mid == HARP_F16) static_cast<__half *>(base)[off] = __float2half_rn(v);
+    else static_cast<float *>(base)[off] = v;
+}
+
 // Load 4 consecutive elements (16-byte f32 or 8-byte bf16 aligned).
 template <int PRO>
 __device__ __forceinline__ void ldg4(const void *base, int64_t off, float (&v)[4]) {
@@ -433,11 +448,12 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const Geo g) {
     // round trips rather than one per element.
     if constexpr (PRO == PRO_CODES) {
         float *lev = X + tile_floats;
-        if (tid < 16) lev[tid] = Q.level[tid];
+        if (tid < 32) lev[tid] = Q.level[tid];
         __syncthreads();
         if (Q.bits == 2) load_codes<2>(X, g, Q, L, lev, v0, tid);
         else if (Q.bits == 3) load_codes<3>(X, g, Q, L, lev, v0, tid);
-        else load_codes<4>(X, g, Q, L, lev, v0, tid);
+        else if (Q.bits == 4) load_codes<4>(X, g, Q, L, lev, v0, tid);
+        else load_codes<5>(X, g, Q, L, lev, v0, tid);
     } else if constexpr (SIDE == SIDE_ROWS) {
         if (VW == 4 && (d & 3) == 0) {
             constexpr int IB = 4;
@@ -618,8 +634,8 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const Geo g) {
                 }
             }
         }
-    } else {
-        // EPI_QUANT / EPI_QUANT_F32: rows side, forward. g % 32 == 0, g | d.
+    } else if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
+        // rows side, forward. g % 32 == 0, g | d.
         const int ng = d / Q.group;
         float *sc = X + tile_floats;                      // [R][ng] stored scale
         float *isc = sc + R * ng;                         // [R][ng] its reciprocal
@@ -627,7 +643,31 @@ vec_kernel(const PlanDev P, const QuantDev Q, const VecLaunch L, const Geo g) {
         constexpr bool F32OUT = (EPI == EPI_QUANT_F32);
         if (Q.bits == 2) quantize_tile<VW, 2, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
         else if (Q.bits == 3) quantize_tile<VW, 3, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
-        else quantize_tile<VW, 4, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
+        else if (Q.bits == 4) quantize_tile<VW, 4, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
+        else quantize_tile<VW, 5, F32OUT>(X, g, Q, sc, isc, L, v0, warp, lane);
+    } else {
+        // EPI_REQUANT: rows side, inverse, codes in. The tile holds the rows
+        // rotated back; apply the inverse signs, round each value to the
+        // restored weights' storage type (optionally stored), then quantise
+        // them with the second codebook. The level table the prologue used
+        // sits where the scales go; the stages' barriers ordered its last read.
+        for (int idx = tid; idx < R * d; idx += NT) {
+            const int r = idx / d, i = idx - r * d;
+            const int64_t row = v0 + r;
+            const float v = round_mid(X[g.row(i) + r] * __ldg(signs + i), L.mid);
+            X[g.row(i) + r] = v;
+            if (L.out && row < nvec) store_mid(L.out, row * L.ld_out + i, v, L.mid);
+        }
+        __syncthreads();
+        const QuantDev &Q2 = L.q2;
+        const int ng = d / Q2.group;
+        float *sc = X + tile_floats;
+        float *isc = sc + R * ng;
+        const int warp = tid >> 5, lane = tid & 31;
+        if (Q2.bits == 2) quantize_tile<VW, 2, false>(X, g, Q2, sc, isc, L, v0, warp, lane);
+        else if (Q2.bits == 3) quantize_tile<VW, 3, false>(X, g, Q2, sc, isc, L, v0, warp, lane);
+        else if (Q2.bits == 4) quantize_tile<VW, 4, false>(X, g, Q2, sc, isc, L, v0, warp, lane);
+        else quantize_tile<VW, 5, false>(X, g, Q2, sc, isc, L, v0, warp, lane);
     }
 }
 
@@ -724,8 +764,8 @@ int64_t smem_floats(const PlanDev &plan, const TileChoice &t, int epi, int pro, 
     const int64_t d = plan.d;
     const int bl = last_radix(plan);
     int64_t f = d * t.R + static_cast<int64_t>(t.VW) * ((d - 1) / bl);
-    if (epi == EPI_QUANT || epi == EPI_QUANT_F32) f += 2 * t.R * (d / group);
-    if (pro == PRO_CODES) f += 16;
+    if (epi == EPI_QUANT || epi == EPI_QUANT_F32 || epi == EPI_REQUANT) f += 2 * t.R * (d / group);
+    if (pro == PRO_CODES) f += 32;
     return f;
 }
 
@@ -754,6 +794,7 @@ KernelFn select_pe(int pro, int epi) {
         if (pro == PRO_CODES) {
             if (epi == EPI_F32) return get_kernel<SIDE, VW, NV, PRO_CODES, EPI_F32>();
             if (epi == EPI_BF16) return get_kernel<SIDE, VW, NV, PRO_CODES, EPI_BF16>();
+            if (epi == EPI_REQUANT) return get_kernel<SIDE, VW, NV, PRO_CODES, EPI_REQUANT>();
             return nullptr;
         }
 #define HARP_ROW_CASE(P)                                                              \
@@ -790,13 +831,14 @@ KernelFn select_tile(int ti, int pro, int epi) {
 
 }  // namespace
 
-int vec_tile(const PlanDev &plan, int epi, int group) {
-    const int ti = pick_tile(plan, epi, PRO_F32, group > 0 ? group : 32);
+int vec_tile(const PlanDev &plan, int epi, int group, int pro) {
+    const int ti = pick_tile(plan, epi, pro, group > 0 ? group : 32);
     return ti < 0 ? 0 : kTiles[ti].R;
 }
 
 int launch_vec(const PlanDev &plan, const QuantDev *q, const VecLaunch &L, void *stream) {
-    const int group = q ? q->group : 32;
+    // the group that sizes the epilogue's scale arrays
+    const int group = (L.epi == EPI_REQUANT) ? L.q2.group : (q ? q->group : 32);
     const int ti = pick_tile(plan, L.epi, L.pro, group);
     if (ti < 0) return static_cast<int>(cudaErrorInvalidValue);
     KernelFn fn = (L.side == HARP_RIGHT) ? select_tile<SIDE_ROWS>(ti, L.pro, L.epi)
@@ -824,11 +866,13 @@ int launch_quantize(const QuantDev &q, const void *in, int in_dtype, int64_t row
     if (in_dtype == HARP_F32) {
         if (q.bits == 2) HARP_QLAUNCH(PRO_F32, 2);
         else if (q.bits == 3) HARP_QLAUNCH(PRO_F32, 3);
-        else HARP_QLAUNCH(PRO_F32, 4);
+        else if (q.bits == 4) HARP_QLAUNCH(PRO_F32, 4);
+        else HARP_QLAUNCH(PRO_F32, 5);
     } else {
         if (q.bits == 2) HARP_QLAUNCH(PRO_BF16, 2);
         else if (q.bits == 3) HARP_QLAUNCH(PRO_BF16, 3);
-        else HARP_QLAUNCH(PRO_BF16, 4);
+        else if (q.bits == 4) HARP_QLAUNCH(PRO_BF16, 4);
+        else HARP_QLAUNCH(PRO_BF16, 5);
     }
 #undef HARP_QLAUNCH
     return static_cast<int>(cudaGetLastError());

@@ -78,7 +78,10 @@ def test_plan_create_without_device_is_a_cuda_error(cuda_available):
 
 def test_codebook_checks_and_tables():
     with pytest.raises(harp.HarpError) as e:
-        harp.Codebook("lloyd_max", 5, 128)
+        harp.Codebook("lloyd_max", 6, 128)
+    assert e.value.status == 3
+    with pytest.raises(harp.HarpError) as e:
+        harp.Codebook("absmax", 1, 128)
     assert e.value.status == 3
     with pytest.raises(harp.HarpError) as e:
         harp.Codebook("lloyd_max", 3, 100)       # group not a multiple of 32
@@ -91,7 +94,7 @@ def test_codebook_checks_and_tables():
     np.testing.assert_array_equal(c, np.arange(16) - 8)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
 def test_library_lloyd_max_table_equals_oracle(bits):
     """The library solves the Lloyd-Max conditions itself (positive half,
     different start); its fp32 table must be the oracle's rounded table."""
@@ -183,3 +186,5 @@ def test_theta_calls_reject_bad_arguments_before_launch():
     assert L.harp_theta_blocks(4, 0, None, 0.01, None, None, None) == 0
     # NULL plan
     assert L.harp_plan_load_theta(None, 0, fake, 0.01, None, None) == 1
+    # two-stage codec: NULL plan or codebooks
+    assert L.harp_requantize(None, None, None, None, 1, 128, 2, None, None, None, None, None) == 1

@@ -275,7 +275,8 @@ def test_small_rotate_both_directions(radix, side):
 
 @pytest.mark.parametrize("kind,bits,group", [("lloyd_max", 2, 32), ("lloyd_max", 3, 64),
                                              ("lloyd_max", 4, 128), ("absmax", 2, 64),
-                                             ("absmax", 3, 512), ("absmax", 4, 32)])
+                                             ("absmax", 3, 512), ("absmax", 4, 32),
+                                             ("lloyd_max", 5, 128), ("absmax", 5, 64)])
 def test_standalone_quantize_and_dequantize(kind, bits, group):
     rows, cols = 33, 512
     X = synth.small_matrix(bits * 10 + group, rows, cols, outlier_cols=3, scale=0.02)
@@ -377,3 +378,28 @@ def test_hadamard_two_sided_matches_oracle():
     out = harp.dequantize_unrotate(left, right, cb, torch.from_numpy(raw).cuda(),
                                    torch.from_numpy(sc.view(np.int16)).cuda(), rows, cols, torch.float32)
     assert rel_l2(out.cpu().numpy(), ref3) <= TOL_F32
+
+
+def test_mixed_radix_5120_two_sided():
+    """HARP section 2.1's arbitrary-d example, 5120 = 8 * 8 * 8 * 5 * 2, as
+    the column processor of a 5120 x 1280 weight (row processor (5, 16, 16)),
+    random orthogonal blocks: the fused forward with 3-bit Lloyd-Max g128 and
+    the inverse of its codes against the oracle, element by element."""
+    left_s = synth.side_draws(31, (8, 8, 8, 5, 2), "qr", synth.S_SIGNS_L, synth.S_BLOCKS_L)
+    right_s = synth.side_draws(31, (5, 16, 16), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    rows, cols = 5120, 1280
+    W = synth.small_matrix(32, rows, cols, outlier_cols=6, scale=0.02)
+    Wb = synth.to_bf16_bits(W)
+    Pl, Pr = oracle.processor(left_s), oracle.processor(right_s)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(synth.bf16_bits_to_f64(Wb), Pl, Pr, "lloyd_max", 3, 128)
+    left, right = harp.Plan.from_side(left_s), harp.Plan.from_side(right_s)
+    cb = harp.Codebook("lloyd_max", 3, 128)
+    xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, rot = harp.rotate_quantize(left, right, cb, xb, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, 3, 128)
+    ref_inv = oracle.dequantize_unrotate(np_unpack(codes.cpu().numpy(), 3, cols), scales_np(scales),
+                                         Pl, Pr, "lloyd_max", 3, 128)
+    out = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.float32)
+    assert rel_l2(out.cpu().numpy(), ref_inv) <= TOL_F32
+
