@@ -578,6 +578,17 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
     if (!aligned(in, 16) || !aligned(codes, 4) || !aligned(scales, 2) ||
         (rotated_out && !aligned(rotated_out, 16)) || cols % 4)
         return HARP_ERR_ALIGNMENT;
+    if (!left && in_dtype == HARP_BF16 && harp::short_ok(right->dev, harp::SHORT_FWD, 0)) {
+        harp::ShortLaunch S{};
+        S.mode = harp::SHORT_FWD;
+        S.nvec = rows;
+        S.in = in;
+        S.out = rotated_out;
+        S.out_dtype = HARP_F32;
+        S.codes = codes;
+        S.scales = scales;
+        return cuda_status(harp::launch_short(right->dev, cb->q, S, stream));
+    }
     if (use_passes(left, right, cb))
         return cuda_status(harp::launch_pass_fwd(left->dev, right->dev, cb->q, in, in_dtype, codes, scales,
                                                  rotated_out, static_cast<float *>(workspace), stream));
@@ -632,6 +643,20 @@ int harp_requantize(harp_plan_t right, harp_codebook_t cb_in, const uint8_t *cod
     if (!aligned(codes_in, 4) || !aligned(scales_in, 2) || !aligned(codes_out, 4) ||
         !aligned(scales_out, 2) || (restored_out && !aligned(restored_out, 16)))
         return HARP_ERR_ALIGNMENT;
+    if (harp::short_ok(right->dev, harp::SHORT_REQUANT, cb_in->q.bits)) {
+        harp::ShortLaunch S{};
+        S.mode = harp::SHORT_REQUANT;
+        S.nvec = rows;
+        S.in_codes = codes_in;
+        S.in_scales = scales_in;
+        S.out = restored_out;
+        S.out_dtype = mid_dtype;
+        S.codes = codes_out;
+        S.scales = scales_out;
+        S.q2 = cb_out->q;
+        S.mid = mid_dtype;
+        return cuda_status(harp::launch_short(right->dev, cb_in->q, S, stream));
+    }
     harp::VecLaunch L{};
     L.side = HARP_RIGHT;
     L.dir = HARP_INV;
@@ -679,6 +704,16 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
     if (rows == 0 || cols == 0) return HARP_OK;
     if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
     if (!aligned(out, 16) || !aligned(scales, 2) || cols % 4) return HARP_ERR_ALIGNMENT;
+    if (!left && harp::short_ok(right->dev, harp::SHORT_INV, cb->q.bits)) {
+        harp::ShortLaunch S{};
+        S.mode = harp::SHORT_INV;
+        S.nvec = rows;
+        S.in_codes = codes;
+        S.in_scales = scales;
+        S.out = out;
+        S.out_dtype = out_dtype;
+        return cuda_status(harp::launch_short(right->dev, cb->q, S, stream));
+    }
     if (use_passes(left, right, cb))
         return cuda_status(harp::launch_pass_inv(left->dev, right->dev, cb->q, codes, scales, out, out_dtype,
                                                  static_cast<float *>(workspace), stream));

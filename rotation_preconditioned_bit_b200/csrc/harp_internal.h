@@ -124,6 +124,28 @@ size_t theta_smem_bytes(int b);
 int launch_theta_blocks(int b, int64_t n_groups, const int8_t *theta, double scale,
                         const float *base, const ThetaOut &o, void *stream);
 
+// Short-vector kernel (harp_short.cu): row-side calls with d = 32, 64 or
+// 128, one thread per vector. Modes: forward (bf16 rows -> codes + scales,
+// optional fp32 rotated copy in `out`), inverse (codes -> rows in
+// out_dtype), requantize (codes -> restored rows in `mid` (optionally
+// stored in `out`) -> codes + scales of q2).
+enum ShortMode { SHORT_FWD = 0, SHORT_INV = 1, SHORT_REQUANT = 2 };
+struct ShortLaunch {
+    int mode;
+    int64_t nvec;
+    const void *in;              // SHORT_FWD: bf16 [nvec][d]
+    const uint8_t *in_codes;     // SHORT_INV / SHORT_REQUANT
+    const uint16_t *in_scales;
+    void *out;                   // optional except SHORT_INV
+    int out_dtype;               // HARP_F32 | HARP_BF16 | HARP_F16
+    uint8_t *codes;              // SHORT_FWD / SHORT_REQUANT outputs
+    uint16_t *scales;
+    QuantDev q2;                 // SHORT_REQUANT: the second quantizer
+    int mid;                     // SHORT_REQUANT: restored storage type
+};
+bool short_ok(const PlanDev &P, int mode, int in_bits);
+int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &L, void *stream);
+
 // Vectors per CTA the whole-vector kernel uses for this plan and epilogue
 // (0 if a vector does not fit in shared memory).
 int vec_tile(const PlanDev &plan, int epi, int group, int pro = PRO_F32);

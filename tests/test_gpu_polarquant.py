@@ -168,3 +168,43 @@ def test_two_sided_q5_takes_the_whole_vector_path():
     ref_back = oracle.dequantize_unrotate(np_unpack(codes.cpu().numpy(), 5, 1024), scales_np(scales),
                                           Pl, Pr, "lloyd_max", 5, 128)
     assert rel_l2(back.cpu().numpy(), ref_back) <= TOL_F32
+
+
+@pytest.mark.parametrize("radix,bits,group", [((4, 8), 4, 32), ((8, 8), 3, 64), ((2, 16, 4), 2, 32)])
+def test_short_vectors_all_three_calls(radix, bits, group):
+    """Rows of 32, 64 and 128 coordinates (one thread per row in the
+    short-vector kernel), 1000 rows (a ragged last tile of 256), random
+    orthogonal blocks with signs: forward (bf16 in, fp32 rotated copy),
+    inverse to bf16, and the two-stage codec to 4-bit absmax."""
+    torch.cuda.set_device(0)
+    side = synth.side_draws(101 + bits, radix, "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    plan, P = harp.Plan.from_side(side), oracle.processor(side)
+    d, rows = int(np.prod(radix)), 1000
+    Wb = bf16_matrix(102 + bits, rows, d)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(synth.bf16_bits_to_f64(Wb), None, P, "lloyd_max", bits, group)
+    cb = harp.Codebook("lloyd_max", bits, group)
+    xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, rot = harp.rotate_quantize(None, plan, cb, xb, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+    raw, sc = synth.random_code_stream(103, rows, d, bits, group)
+    ref_inv = oracle.dequantize_unrotate(oracle.unpack(bits, raw, d), sc, None, P, "lloyd_max", bits, group)
+    out = harp.dequantize_unrotate(None, plan, cb, torch.from_numpy(raw).cuda(),
+                                   torch.from_numpy(sc.view(np.int16)).cuda(), rows, d, torch.bfloat16)
+    assert rel_l2(out.float().cpu().numpy(), ref_inv) <= 1e-2
+    got, Y, codes_out, scales_out = _requant_case_g(plan, P, raw, sc, rows, d, bits, group)
+    assert_restored_match(got, Y, "f16")
+    oc2, osc2, m2, sm2 = oracle.quantize("absmax", 4, 32, got)
+    compare_quant(codes_out.cpu().numpy(), scales_np(scales_out), oc2, osc2, m2, sm2, 4, 32)
+
+
+def _requant_case_g(plan, P, raw, sc, rows, d, bits, group):
+    cb_in = harp.Codebook("lloyd_max", bits, group)
+    cb_out = harp.Codebook("absmax", 4, 32)
+    codes_out, scales_out = harp.empty_codes(rows, d, cb_out)
+    restored = torch.empty((rows, d), dtype=torch.float16, device="cuda")
+    harp.harp_requantize(plan, cb_in, torch.from_numpy(raw).cuda(), torch.from_numpy(sc.view(np.int16)).cuda(),
+                         rows, d, "f16", cb_out, codes_out, scales_out, restored)
+    torch.cuda.synchronize()
+    Y = oracle.requantize(oracle.unpack(bits, raw, d), sc, P, "lloyd_max", bits, group, "f16", "absmax", 4, 32)[0]
+    return restored.float().cpu().numpy().astype(np.float64), Y, codes_out, scales_out
