@@ -142,6 +142,7 @@ struct ShortLaunch {
     uint16_t *scales;
     QuantDev q2;                 // SHORT_REQUANT: the second quantizer
     int mid;                     // SHORT_REQUANT: restored storage type
+    int bins;                    // set by launch_short: binned Lloyd-Max code search
 };
 bool short_ok(const PlanDev &P, int mode, int in_bits);
 int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &L, void *stream);

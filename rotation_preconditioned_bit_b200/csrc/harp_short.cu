@@ -22,6 +22,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
+
 #include "harp_internal.h"
 #include "harp_quant_dev.cuh"
 
@@ -61,7 +63,7 @@ struct ShortLayout {
     int coef_off, coef_words;
     int coef_total;  // words of all stages' blocks (coef_words rounds it up)
     int sign_off;    // d words
-    int tab_off;     // 32 levels, then 32 thresholds
+    int tab_off;     // 32 levels, 32 thresholds (+inf past the last), 256 bin bytes
     int stage_off;   // staging buffer
     int stage_pitch; // words per staged row
     int total_words;
@@ -79,7 +81,7 @@ __host__ __device__ inline ShortLayout short_layout(const PlanDev &P, int mode, 
     L.coef_words = (cw + 3) & ~3;
     L.sign_off = L.coef_off + L.coef_words;
     L.tab_off = L.sign_off + ((d + 3) & ~3);
-    L.stage_off = L.tab_off + 64;
+    L.stage_off = L.tab_off + 64 + 64;
     // bf16 rows: d/2 words padded to a multiple of 4 plus 4 (16-byte rows
     // whose 16-byte reads by 8 neighbouring lanes cover all 32 banks);
     // codes: d*bits/32 words rounded up to an odd count (conflict-free
@@ -168,10 +170,26 @@ __device__ __forceinline__ void run_stage_row(float *xr, const float *C, const S
     else stage_row<64>(xr, C, b, kp, s, d);
 }
 
+// Lloyd-Max code = number of midpoints t_k below z, found with one table
+// read and one compare: bin = rint(32 z + 128) clamped to [0, 255] (a single
+// rounding of an exact product-sum: z lies in [(bin - 128.5)/32,
+// (bin - 127.5)/32] unless clamped), bins[bin] = number of midpoints below
+// the bin's lower edge (0 for bin 0), and the host has checked that no bin
+// holds two midpoints (the edge bins included, open-ended), so the code is
+// bins[bin] or one more. thr[K - 1] is +inf.
+__device__ __forceinline__ int code_binned(float z, const float *thr, const unsigned char *bins) {
+    const float y = fmaf(z, 32.0f, 128.0f + 12582912.0f);     // 12582912 = 1.5 * 2^23
+    int bin = __float_as_int(y) - 0x4B400000;
+    bin = min(max(bin, 0), 255);
+    const int c = bins[bin];
+    return c + ((z > thr[c]) ? 1 : 0);
+}
+
 // Quantise one row in place: scales to global, packed words into the row's
 // own shared memory (chunk k of 32 codes -> words [k*BITS, k*BITS + BITS)).
 template <int BITS>
-__device__ __forceinline__ void quantize_row(float *xr, const QuantDev &Q, const float *thr, int d,
+__device__ __forceinline__ void quantize_row(float *xr, const QuantDev &Q, const float *thr,
+                                             const unsigned char *bins, bool use_bins, int d,
                                              uint16_t *scales_row) {
     const int g = Q.group, ngr = d / g;
     const bool is_max = (Q.kind == HARP_ABSMAX);
@@ -193,7 +211,9 @@ __device__ __forceinline__ void quantize_row(float *xr, const QuantDev &Q, const
             for (int i = 0; i < BITS; ++i) w[i] = 0u;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const unsigned code = static_cast<unsigned>(code_of_smem<BITS>(v[e], s, inv, !is_max, thr));
+                const unsigned code = static_cast<unsigned>(
+                    (use_bins && s > 0.0f) ? code_binned(v[e] * inv, thr, bins)
+                                           : code_of_smem<BITS>(v[e], s, inv, !is_max, thr));
                 const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
                 w[wi] |= code << sh;
                 if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
@@ -255,6 +275,7 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
     float *sg = sm + Y.sign_off;
     float *lev = sm + Y.tab_off;
     float *thr = lev + 32;
+    unsigned char *bins = reinterpret_cast<unsigned char *>(lev + 64);
     unsigned *stg = reinterpret_cast<unsigned *>(sm + Y.stage_off);
     const bool fwd = (MODE == SHORT_FWD);
     const QuantDev &QO = (MODE == SHORT_REQUANT) ? L.q2 : Q;   // the quantizer of the epilogue
@@ -270,9 +291,18 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             off += n4 * 4;
         }
         for (int i = tid; i < d; i += ST) sg[i] = __ldg(P.signs + i);
+        const int K = 1 << QO.bits;
         if (tid < 32) {
             lev[tid] = Q.level[tid];
-            thr[tid] = QO.thr[tid];
+            thr[tid] = (tid < K - 1) ? QO.thr[tid] : __int_as_float(0x7f800000);
+        }
+        if (L.bins) {
+            // bins[i] = number of midpoints below (i - 128.5) / 32; bin 0 open below
+            const float lo = (static_cast<float>(tid) - 128.5f) * 0.03125f;
+            int c = 0;
+            if (tid > 0)
+                for (int k = 0; k < K - 1; ++k) c += (QO.thr[k] < lo) ? 1 : 0;
+            bins[tid] = static_cast<unsigned char>(c);
         }
     }
 
@@ -370,14 +400,24 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
         void *vout = L.out;
         if (vout) {
             __syncthreads();
-            const int odt = L.out_dtype;
-            for (int i = tid; i < nv * d; i += ST) {
-                const int r = i >> ld, c = i & (d - 1);
-                const float v = X[r * Y.xp + c];
-                const int64_t off = (v0 + r) * d + c;
-                if (odt == HARP_F32) static_cast<float *>(vout)[off] = v;
-                else if (odt == HARP_BF16) static_cast<unsigned short *>(vout)[off] = f_to_bf16(v);
-                else static_cast<__half *>(vout)[off] = __float2half_rn(v);
+            // one warp per row, each lane a pair of neighbouring columns:
+            // 32-bit stores of two 16-bit values, 64-bit stores of two floats
+            const int odt = L.out_dtype, lane = tid & 31;
+            for (int r = tid >> 5; r < nv; r += ST / 32) {
+                const float *xs = X + r * Y.xp;
+                const int64_t off = (v0 + r) * d;
+                for (int c = 2 * lane; c < d; c += 64) {
+                    const float a = xs[c], b = xs[c + 1];
+                    if (odt == HARP_F32) {
+                        *reinterpret_cast<float2 *>(static_cast<float *>(vout) + off + c) = make_float2(a, b);
+                    } else if (odt == HARP_BF16) {
+                        *reinterpret_cast<unsigned *>(static_cast<unsigned short *>(vout) + off + c) =
+                            f_to_bf16(a) | (static_cast<unsigned>(f_to_bf16(b)) << 16);
+                    } else {
+                        *reinterpret_cast<__half2 *>(static_cast<__half *>(vout) + off + c) =
+                            __halves2half2(__float2half_rn(a), __float2half_rn(b));
+                    }
+                }
             }
         }
         if constexpr (MODE != SHORT_INV) {
@@ -385,10 +425,10 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             if (mine) {
                 uint16_t *srow = L.scales + (v0 + tid) * (d / QO.group);
                 switch (QO.bits) {
-                    case 2: quantize_row<2>(xr, QO, thr, d, srow); break;
-                    case 3: quantize_row<3>(xr, QO, thr, d, srow); break;
-                    case 4: quantize_row<4>(xr, QO, thr, d, srow); break;
-                    default: quantize_row<5>(xr, QO, thr, d, srow); break;
+                    case 2: quantize_row<2>(xr, QO, thr, bins, L.bins, d, srow); break;
+                    case 3: quantize_row<3>(xr, QO, thr, bins, L.bins, d, srow); break;
+                    case 4: quantize_row<4>(xr, QO, thr, bins, L.bins, d, srow); break;
+                    default: quantize_row<5>(xr, QO, thr, bins, L.bins, d, srow); break;
                 }
             }
             __syncthreads();
@@ -414,8 +454,27 @@ bool short_ok(const PlanDev &P, int mode, int in_bits) {
     return short_smem_bytes(P, mode, in_bits) <= SMEM_LIMIT;
 }
 
-int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &L, void *stream) {
-    if (L.nvec == 0) return cudaSuccess;
+// Whether the bin table of code_binned is exact for these midpoints: no bin
+// [(i - 128.5)/32, (i - 127.5)/32) (bin 0 open below, bin 255 open above)
+// holds two of them.
+bool bins_exact(const QuantDev &q) {
+    if (q.kind != HARP_LLOYD_MAX) return false;
+    const int K = 1 << q.bits;
+    int prev_bin = -1;
+    for (int k = 0; k < K - 1; ++k) {
+        const double t = static_cast<double>(q.thr[k]);
+        int bin = static_cast<int>(std::floor((t * 32.0 + 128.5)));   // t in [lo_bin, lo_bin + 1/32)
+        bin = bin < 0 ? 0 : (bin > 255 ? 255 : bin);
+        if (bin == prev_bin) return false;
+        prev_bin = bin;
+    }
+    return true;
+}
+
+int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &Lin, void *stream) {
+    if (Lin.nvec == 0) return cudaSuccess;
+    ShortLaunch L = Lin;
+    L.bins = (L.mode == SHORT_INV) ? 0 : (bins_exact(L.mode == SHORT_REQUANT ? L.q2 : q) ? 1 : 0);
     const int in_bits = (L.mode == SHORT_FWD) ? 0 : q.bits;
     const size_t smem = short_smem_bytes(P, L.mode, in_bits);
     const void *fn = (L.mode == SHORT_FWD) ? reinterpret_cast<const void *>(short_kernel<SHORT_FWD>)
