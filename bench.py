@@ -298,7 +298,10 @@ def run_gpu(args, rank, world, local_rank):
     return total_ms, step_ms, kt, clk, e2e, npass, pass_fma
 
 
-def run_workloads(steps, dev):
+WORKLOAD_NAMES = ("c1", "c3", "c4", "c5", "rht", "pq", "theta")
+
+
+def run_workloads(steps, dev, names=WORKLOAD_NAMES):
     """The other synthetic workloads, through the public calls with inputs
     resident on the device: per call, mean device time over `steps` calls
     (CUDA events; L2 not flushed: each call streams more than L2 except c1),
@@ -323,7 +326,7 @@ def run_workloads(steps, dev):
         return a.elapsed_time(b) / steps * 1e-3
 
     out = {}
-    for name in ("c1", "c3", "c4", "c5", "rht"):
+    for name in [n for n in ("c1", "c3", "c4", "c5", "rht") if n in names]:
         if name == "rht":
             # the c2 weight with Hadamard-initialised processors on both sides
             # (random signs, normalised Sylvester blocks: HARP's theta = 0 start)
@@ -362,8 +365,10 @@ def run_workloads(steps, dev):
             out[key] = rec
         del x, ws
         torch.cuda.empty_cache()
-    out.update(run_polarquant(timed, dev))
-    out.update(run_theta_loads(timed, dev))
+    if "pq" in names:
+        out.update(run_polarquant(timed, dev))
+    if "theta" in names:
+        out.update(run_theta_loads(timed, dev))
     return out
 
 
@@ -556,7 +561,19 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--workloads", action="store_true",
                     help="also time the c1, c3, c4 and c5 workloads (adds ~1 min of input generation)")
+    ap.add_argument("--workloads-only", default=None, metavar="NAMES",
+                    help="time only these workloads (comma list of " + ",".join(WORKLOAD_NAMES) +
+                         ") on one GPU, print them as one JSON line and exit")
     args = ap.parse_args()
+    if args.workloads_only is not None:
+        import torch
+        names = tuple(n for n in args.workloads_only.split(",") if n)
+        bad = [n for n in names if n not in WORKLOAD_NAMES]
+        if bad:
+            ap.error(f"unknown workloads {bad}")
+        torch.cuda.set_device(0)
+        print(json.dumps({"workloads": run_workloads(max(3, args.steps), torch.device("cuda", 0), names)}))
+        return
     args.warmup = max(3, args.warmup)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
