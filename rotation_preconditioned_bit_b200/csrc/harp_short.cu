@@ -32,8 +32,12 @@ namespace {
 
 using namespace dq;
 
-constexpr int ST = 256;        // threads per CTA = vectors per tile
+constexpr int ST = 256;        // vectors per tile
+constexpr int NP = 2;          // threads per vector
+constexpr int NTT = ST * NP;   // threads per CTA
 constexpr int SD_MAX = 128;    // longest vector handled here
+constexpr int B_MAX = 32;      // largest radix handled here (registers)
+constexpr int MAXCH = SD_MAX / 32 / NP;   // 32-code chunks of a row per thread
 constexpr size_t SMEM_LIMIT = 232448;
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
@@ -64,6 +68,7 @@ struct ShortLayout {
     int coef_total;  // words of all stages' blocks (coef_words rounds it up)
     int sign_off;    // d words
     int tab_off;     // 32 levels, 32 thresholds (+inf past the last), 256 bin bytes
+    int red_off;     // [NP][4][ST] partial group statistics
     int stage_off;   // staging buffer
     int stage_pitch; // words per staged row
     int total_words;
@@ -81,7 +86,8 @@ __host__ __device__ inline ShortLayout short_layout(const PlanDev &P, int mode, 
     L.coef_words = (cw + 3) & ~3;
     L.sign_off = L.coef_off + L.coef_words;
     L.tab_off = L.sign_off + ((d + 3) & ~3);
-    L.stage_off = L.tab_off + 64 + 64;
+    L.red_off = L.tab_off + 64 + 64;
+    L.stage_off = L.red_off + NP * 4 * ST;
     // bf16 rows: d/2 words padded to a multiple of 4 plus 4 (16-byte rows
     // whose 16-byte reads by 8 neighbouring lanes cover all 32 banks);
     // codes: d*bits/32 words rounded up to an odd count (conflict-free
@@ -123,11 +129,13 @@ __device__ __forceinline__ const float *stage_cols(const StageDev &S, bool fwd) 
 // packed pairs, input by input, so consecutive FMAs are independent.
 // BM >= max(b, 4) is the register width; padding coefficients are zero.
 template <int BM>
-__device__ __forceinline__ void stage_row(float *xr, const float *C, int b, int kpad, int s, int d) {
+__device__ __forceinline__ void stage_row(float *xr, const float *C, int b, int kpad, int s, int d, int part) {
     const int nh = d / (b * s);
-    const float *cr = C;
+    int cidx = 0;
     for (int h = 0; h < nh; ++h) {
-        for (int l = 0; l < s; ++l, cr += b * kpad) {
+        for (int l = 0; l < s; ++l, ++cidx) {
+            if ((cidx & (NP - 1)) != part) continue;      // the row's groups alternate between its threads
+            const float *cr = C + cidx * b * kpad;
             float *base = xr + h * b * s + l;
             float x[BM];
 #pragma unroll
@@ -161,13 +169,12 @@ __device__ __forceinline__ void stage_row(float *xr, const float *C, int b, int 
     }
 }
 
-__device__ __forceinline__ void run_stage_row(float *xr, const float *C, const StageDev &S, int d) {
+__device__ __forceinline__ void run_stage_row(float *xr, const float *C, const StageDev &S, int d, int part) {
     const int b = S.b, kp = S.kpad, s = static_cast<int>(S.s);
-    if (b <= 4) stage_row<4>(xr, C, b, kp, s, d);
-    else if (b <= 8) stage_row<8>(xr, C, b, kp, s, d);
-    else if (b <= 16) stage_row<16>(xr, C, b, kp, s, d);
-    else if (b <= 32) stage_row<32>(xr, C, b, kp, s, d);
-    else stage_row<64>(xr, C, b, kp, s, d);
+    if (b <= 4) stage_row<4>(xr, C, b, kp, s, d, part);
+    else if (b <= 8) stage_row<8>(xr, C, b, kp, s, d, part);
+    else if (b <= 16) stage_row<16>(xr, C, b, kp, s, d, part);
+    else stage_row<B_MAX>(xr, C, b, kp, s, d, part);
 }
 
 // Lloyd-Max code = number of midpoints t_k below z, found with one table
@@ -185,51 +192,94 @@ __device__ __forceinline__ int code_binned(float z, const float *thr, const unsi
     return c + ((z > thr[c]) ? 1 : 0);
 }
 
-// Quantise one row in place: scales to global, packed words into the row's
-// own shared memory (chunk k of 32 codes -> words [k*BITS, k*BITS + BITS)).
+// One of the 4 values a[0..3] picked by a runtime index (registers only).
+__device__ __forceinline__ float pick4(const float (&a)[4], int i) {
+    return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+}
+
+// Quantise the tile's rows; thread (v, part) owns chunks part, part + NP, ...
+// of row v (32 codes each). Group statistics: each thread sums (or maxes)
+// its chunks of every group in order, the NP partials meet in shared memory
+// and are combined in part order. Codes are formed in registers; after a
+// barrier (every value of the row has been read) the packed words of chunk k
+// go to words [k*BITS, k*BITS + BITS) of the row's own shared memory.
+// Called by every thread of the CTA (it holds barriers).
 template <int BITS>
-__device__ __forceinline__ void quantize_row(float *xr, const QuantDev &Q, const float *thr,
-                                             const unsigned char *bins, bool use_bins, int d,
-                                             uint16_t *scales_row) {
-    const int g = Q.group, ngr = d / g;
+__device__ __forceinline__ void quantize_rows(float *xr, const QuantDev &Q, const float *thr,
+                                              const unsigned char *bins, bool use_bins, int d, int part,
+                                              float *red, int v, bool mine, uint16_t *scales_row) {
+    const int g = Q.group, ngr = d / g, nch = d / 32, lcpg = __ffs(g / 32) - 1;
     const bool is_max = (Q.kind == HARP_ABSMAX);
-    for (int q = 0; q < ngr; ++q) {
-        const float *gp = xr + q * g;
-        float st = 0.0f;
-        for (int i = 0; i < g; ++i) st = combine(st, gp[i], is_max);
-        const unsigned short hb = group_scale_bits(st, Q);
-        scales_row[q] = hb;
-        const float s = __half2float(__ushort_as_half(hb));
-        const float inv = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
-        for (int k = 0; k < g / 32; ++k) {
-            const int ck = (q * g) / 32 + k;       // chunk index within the row
-            float v[32];
+    float st[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = xr[ck * 32 + e];
-            unsigned w[BITS];
+    for (int ci = 0; ci < MAXCH; ++ci) {
+        const int ck = part + ci * NP;
+        if (mine && ck < nch) {
+            const int q = ck >> lcpg;
+            float a = pick4(st, q);
+            for (int e = 0; e < 32; ++e) a = combine(a, xr[ck * 32 + e], is_max);
 #pragma unroll
-            for (int i = 0; i < BITS; ++i) w[i] = 0u;
+            for (int qq = 0; qq < 4; ++qq)
+                if (qq == q) st[qq] = a;
+        }
+    }
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) red[(part * 4 + qq) * ST + v] = st[qq];
+    __syncthreads();
+    float sc[4] = {0.f, 0.f, 0.f, 0.f}, inv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+        if (mine && qq < ngr) {
+            float tot = red[qq * ST + v];
+#pragma unroll
+            for (int pp = 1; pp < NP; ++pp) {
+                const float o = red[(pp * 4 + qq) * ST + v];
+                tot = is_max ? fmaxf(tot, o) : tot + o;
+            }
+            const unsigned short hb = group_scale_bits(tot, Q);
+            if (part == 0) scales_row[qq] = hb;
+            sc[qq] = __half2float(__ushort_as_half(hb));
+            inv[qq] = (sc[qq] > 0.0f) ? __frcp_rn(sc[qq]) : 0.0f;
+        }
+    }
+    unsigned w[MAXCH][BITS];
+#pragma unroll
+    for (int ci = 0; ci < MAXCH; ++ci) {
+#pragma unroll
+        for (int i = 0; i < BITS; ++i) w[ci][i] = 0u;
+        const int ck = part + ci * NP;
+        if (mine && ck < nch) {
+            const int q = ck >> lcpg;
+            const float s = pick4(sc, q), is = pick4(inv, q);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
+                const float x = xr[ck * 32 + e];
                 const unsigned code = static_cast<unsigned>(
-                    (use_bins && s > 0.0f) ? code_binned(v[e] * inv, thr, bins)
-                                           : code_of_smem<BITS>(v[e], s, inv, !is_max, thr));
+                    (use_bins && s > 0.0f) ? code_binned(x * is, thr, bins)
+                                           : code_of_smem<BITS>(x, s, is, !is_max, thr));
                 const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
-                w[wi] |= code << sh;
-                if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
+                w[ci][wi] |= code << sh;
+                if (sh + BITS > 32) w[ci][wi + 1] |= code >> (32 - sh);
             }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ci = 0; ci < MAXCH; ++ci) {
+        const int ck = part + ci * NP;
+        if (mine && ck < nch) {
             unsigned *dst = reinterpret_cast<unsigned *>(xr) + ck * BITS;
 #pragma unroll
-            for (int i = 0; i < BITS; ++i) dst[i] = w[i];
+            for (int i = 0; i < BITS; ++i) dst[i] = w[ci][i];
         }
     }
 }
 
 template <int BITS>
 __device__ __forceinline__ void decode_row(float *xr, const unsigned *src, const float *lev, const float *sc,
-                                           int g, int d) {
+                                           int g, int d, int part) {
     constexpr unsigned MASK = (1u << BITS) - 1u;
-    for (int ch = 0; ch < d / 32; ++ch) {
+    for (int ch = part; ch < d / 32; ch += NP) {
         unsigned w[BITS];
 #pragma unroll
         for (int i = 0; i < BITS; ++i) w[i] = src[ch * BITS + i];
@@ -255,18 +305,19 @@ __device__ __forceinline__ void store_codes(const float *X, int xp, int d, int64
     unsigned *dst = reinterpret_cast<unsigned *>(codes) + v0 * wpr;
     const int n = nv * wpr;
     const int dk = d / 32;
-    for (int i = tid; i < n; i += ST) {
+    for (int i = tid; i < n; i += NTT) {
         const int r = (i / BITS) / dk, k = i - r * wpr;
         dst[i] = reinterpret_cast<const unsigned *>(X)[r * xp + k];
     }
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(ST, 1)
+__global__ void __launch_bounds__(NTT, 1)
 short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
     extern __shared__ float4 smem_f4[];
     float *sm = reinterpret_cast<float *>(smem_f4);
     const int tid = threadIdx.x;
+    const int v = tid & (ST - 1), part = tid / ST;   // the thread's vector and its share of it
     const int d = static_cast<int>(P.d);
     const int in_bits = (MODE == SHORT_FWD) ? 0 : Q.bits;
     const ShortLayout Y = short_layout(P, MODE, in_bits);
@@ -276,6 +327,7 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
     float *lev = sm + Y.tab_off;
     float *thr = lev + 32;
     unsigned char *bins = reinterpret_cast<unsigned char *>(lev + 64);
+    float *red = sm + Y.red_off;
     unsigned *stg = reinterpret_cast<unsigned *>(sm + Y.stage_off);
     const bool fwd = (MODE == SHORT_FWD);
     const QuantDev &QO = (MODE == SHORT_REQUANT) ? L.q2 : Q;   // the quantizer of the epilogue
@@ -287,16 +339,16 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             const StageDev &S = P.st[t];
             const int n4 = static_cast<int>(d / S.b) * S.b * S.kpad / 4;
             const float4 *src = reinterpret_cast<const float4 *>(stage_cols(S, fwd));
-            for (int i = tid; i < n4; i += ST) reinterpret_cast<float4 *>(C + off)[i] = __ldg(src + i);
+            for (int i = tid; i < n4; i += NTT) reinterpret_cast<float4 *>(C + off)[i] = __ldg(src + i);
             off += n4 * 4;
         }
-        for (int i = tid; i < d; i += ST) sg[i] = __ldg(P.signs + i);
+        for (int i = tid; i < d; i += NTT) sg[i] = __ldg(P.signs + i);
         const int K = 1 << QO.bits;
         if (tid < 32) {
             lev[tid] = Q.level[tid];
             thr[tid] = (tid < K - 1) ? QO.thr[tid] : __int_as_float(0x7f800000);
         }
-        if (L.bins) {
+        if (L.bins && tid < 256) {
             // bins[i] = number of midpoints below (i - 128.5) / 32; bin 0 open below
             const float lo = (static_cast<float>(tid) - 128.5f) * 0.03125f;
             int c = 0;
@@ -319,21 +371,21 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             const int gsh = ld - 3;                       // 16-byte granules per row: d / 8
             const int gpr = 1 << gsh;
             const unsigned short *src = static_cast<const unsigned short *>(L.in);
-            for (int i = tid; i < nv * gpr; i += ST) {
+            for (int i = tid; i < nv * gpr; i += NTT) {
                 const int r = i >> gsh, k = i & (gpr - 1);
                 cp_async16(stg + r * Y.stage_pitch + k * 4, src + (v0 + r) * d + k * 8);
             }
         } else {
             // one warp per row, lanes over the row's words
             const unsigned *src = reinterpret_cast<const unsigned *>(L.in_codes);
-            for (int r = tid >> 5; r < nv; r += ST / 32)
+            for (int r = tid >> 5; r < nv; r += NTT / 32)
                 for (int k = tid & 31; k < wpr_in; k += 32)
                     cp_async4(stg + r * Y.stage_pitch + k, src + (v0 + r) * wpr_in + k);
-            if (tid < nv) {
+            if (v < nv) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     if (q < ng_in)
-                        sc_next[q] = __half2float(__ushort_as_half(__ldg(L.in_scales + (v0 + tid) * ng_in + q)));
+                        sc_next[q] = __half2float(__ushort_as_half(__ldg(L.in_scales + (v0 + v) * ng_in + q)));
             }
         }
         cp_async_commit();
@@ -343,15 +395,15 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int64_t v0 = tile * ST;
         const int nv = (L.nvec - v0 < ST) ? static_cast<int>(L.nvec - v0) : ST;
-        const bool mine = tid < nv;
-        float *xr = X + tid * Y.xp;
+        const bool mine = v < nv;
+        float *xr = X + v * Y.xp;
         cp_async_wait_all();
         __syncthreads();            // staging landed; previous tile's readers of X are done
         float sc[4] = {sc_next[0], sc_next[1], sc_next[2], sc_next[3]};
         if (mine) {
             if constexpr (MODE == SHORT_FWD) {
-                const uint4 *row = reinterpret_cast<const uint4 *>(stg + tid * Y.stage_pitch);
-                for (int k = 0; k < d / 8; ++k) {
+                const uint4 *row = reinterpret_cast<const uint4 *>(stg + v * Y.stage_pitch);
+                for (int k = part; k < d / 8; k += NP) {
                     const uint4 u = row[k];
                     const unsigned w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -361,49 +413,49 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
                     }
                 }
             } else {
-                const unsigned *row = stg + tid * Y.stage_pitch;
+                const unsigned *row = stg + v * Y.stage_pitch;
                 switch (in_bits) {
-                    case 2: decode_row<2>(xr, row, lev, sc, Q.group, d); break;
-                    case 3: decode_row<3>(xr, row, lev, sc, Q.group, d); break;
-                    case 4: decode_row<4>(xr, row, lev, sc, Q.group, d); break;
-                    default: decode_row<5>(xr, row, lev, sc, Q.group, d); break;
+                    case 2: decode_row<2>(xr, row, lev, sc, Q.group, d, part); break;
+                    case 3: decode_row<3>(xr, row, lev, sc, Q.group, d, part); break;
+                    case 4: decode_row<4>(xr, row, lev, sc, Q.group, d, part); break;
+                    default: decode_row<5>(xr, row, lev, sc, Q.group, d, part); break;
                 }
             }
         }
-        __syncthreads();            // staging consumed: the next tile may land in it
+        __syncthreads();            // staging consumed, rows complete
         if (tile + gridDim.x < ntiles) issue(tile + gridDim.x);
 
-        if (mine) {
-            if (fwd) {
-                int o = 0;
-                for (int t = 0; t < P.m; ++t) {
-                    run_stage_row(xr, C + o, P.st[t], d);
-                    o += static_cast<int>(d / P.st[t].b) * P.st[t].b * P.st[t].kpad;
-                }
-            } else {
-                int o = Y.coef_total;
-                for (int t = P.m - 1; t >= 0; --t) {
-                    o -= static_cast<int>(d / P.st[t].b) * P.st[t].b * P.st[t].kpad;
-                    run_stage_row(xr, C + o, P.st[t], d);
+        if (fwd) {
+            int o = 0;
+            for (int t = 0; t < P.m; ++t) {
+                if (mine) run_stage_row(xr, C + o, P.st[t], d, part);
+                __syncthreads();
+                o += static_cast<int>(d / P.st[t].b) * P.st[t].b * P.st[t].kpad;
+            }
+        } else {
+            int o = Y.coef_total;
+            for (int t = P.m - 1; t >= 0; --t) {
+                o -= static_cast<int>(d / P.st[t].b) * P.st[t].b * P.st[t].kpad;
+                if (mine) run_stage_row(xr, C + o, P.st[t], d, part);
+                __syncthreads();
+            }
+            if (mine) {
+                for (int i = part; i < d; i += NP) {
+                    float x = xr[i] * sg[i];
+                    if constexpr (MODE == SHORT_REQUANT) x = round_mid(x, L.mid);
+                    xr[i] = x;
                 }
             }
-            if (!fwd) {
-                for (int i = 0; i < d; ++i) {
-                    float v = xr[i] * sg[i];
-                    if constexpr (MODE == SHORT_REQUANT) v = round_mid(v, L.mid);
-                    xr[i] = v;
-                }
-            }
+            __syncthreads();
         }
 
         // values out (inverse result, rotated copy or restored weights)
         void *vout = L.out;
         if (vout) {
-            __syncthreads();
             // one warp per row, each lane a pair of neighbouring columns:
             // 32-bit stores of two 16-bit values, 64-bit stores of two floats
             const int odt = L.out_dtype, lane = tid & 31;
-            for (int r = tid >> 5; r < nv; r += ST / 32) {
+            for (int r = tid >> 5; r < nv; r += NTT / 32) {
                 const float *xs = X + r * Y.xp;
                 const int64_t off = (v0 + r) * d;
                 for (int c = 2 * lane; c < d; c += 64) {
@@ -421,15 +473,14 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             }
         }
         if constexpr (MODE != SHORT_INV) {
-            if (vout) __syncthreads();
-            if (mine) {
-                uint16_t *srow = L.scales + (v0 + tid) * (d / QO.group);
-                switch (QO.bits) {
-                    case 2: quantize_row<2>(xr, QO, thr, bins, L.bins, d, srow); break;
-                    case 3: quantize_row<3>(xr, QO, thr, bins, L.bins, d, srow); break;
-                    case 4: quantize_row<4>(xr, QO, thr, bins, L.bins, d, srow); break;
-                    default: quantize_row<5>(xr, QO, thr, bins, L.bins, d, srow); break;
-                }
+            // (quantize_rows reads X only after its first barrier; the row
+            // stores above read X too and never write it)
+            uint16_t *srow = L.scales + (v0 + v) * (d / QO.group);
+            switch (QO.bits) {
+                case 2: quantize_rows<2>(xr, QO, thr, bins, L.bins, d, part, red, v, mine, srow); break;
+                case 3: quantize_rows<3>(xr, QO, thr, bins, L.bins, d, part, red, v, mine, srow); break;
+                case 4: quantize_rows<4>(xr, QO, thr, bins, L.bins, d, part, red, v, mine, srow); break;
+                default: quantize_rows<5>(xr, QO, thr, bins, L.bins, d, part, red, v, mine, srow); break;
             }
             __syncthreads();
             switch (QO.bits) {
@@ -451,6 +502,8 @@ size_t short_smem_bytes(const PlanDev &P, int mode, int in_bits) {
 
 bool short_ok(const PlanDev &P, int mode, int in_bits) {
     if (P.d != 32 && P.d != 64 && P.d != SD_MAX) return false;
+    for (int t = 0; t < P.m; ++t)
+        if (P.st[t].b > B_MAX) return false;
     return short_smem_bytes(P, mode, in_bits) <= SMEM_LIMIT;
 }
 
@@ -485,15 +538,15 @@ int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &Lin, vo
     int dev = 0, sms = 0, per_sm = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, ST, smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NTT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t ntiles = (L.nvec + ST - 1) / ST;
     const int64_t grid = ntiles < static_cast<int64_t>(sms) * per_sm ? ntiles : static_cast<int64_t>(sms) * per_sm;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (L.mode == SHORT_FWD) short_kernel<SHORT_FWD><<<static_cast<unsigned>(grid), ST, smem, st>>>(P, q, L);
-    else if (L.mode == SHORT_INV) short_kernel<SHORT_INV><<<static_cast<unsigned>(grid), ST, smem, st>>>(P, q, L);
-    else short_kernel<SHORT_REQUANT><<<static_cast<unsigned>(grid), ST, smem, st>>>(P, q, L);
+    if (L.mode == SHORT_FWD) short_kernel<SHORT_FWD><<<static_cast<unsigned>(grid), NTT, smem, st>>>(P, q, L);
+    else if (L.mode == SHORT_INV) short_kernel<SHORT_INV><<<static_cast<unsigned>(grid), NTT, smem, st>>>(P, q, L);
+    else short_kernel<SHORT_REQUANT><<<static_cast<unsigned>(grid), NTT, smem, st>>>(P, q, L);
     return cudaGetLastError();
 }
 
