@@ -128,8 +128,9 @@ __device__ __forceinline__ const float *stage_cols(const StageDev &S, bool fwd) 
 // one rounding per FMA), written back in place. Outputs are accumulated in
 // packed pairs, input by input, so consecutive FMAs are independent.
 // BM >= max(b, 4) is the register width; padding coefficients are zero.
-template <int BM>
-__device__ __forceinline__ void stage_row(float *xr, const float *C, int b, int kpad, int s, int d, int part) {
+template <int BM, bool EXACT>
+__device__ __forceinline__ void stage_row(float *xr, const float *C, int b_rt, int kpad, int s, int d, int part) {
+    const int b = EXACT ? BM : b_rt;      // b == BM: every guard below folds away
     const int nh = d / (b * s);
     int cidx = 0;
     for (int h = 0; h < nh; ++h) {
@@ -171,10 +172,17 @@ __device__ __forceinline__ void stage_row(float *xr, const float *C, int b, int 
 
 __device__ __forceinline__ void run_stage_row(float *xr, const float *C, const StageDev &S, int d, int part) {
     const int b = S.b, kp = S.kpad, s = static_cast<int>(S.s);
-    if (b <= 4) stage_row<4>(xr, C, b, kp, s, d, part);
-    else if (b <= 8) stage_row<8>(xr, C, b, kp, s, d, part);
-    else if (b <= 16) stage_row<16>(xr, C, b, kp, s, d, part);
-    else stage_row<B_MAX>(xr, C, b, kp, s, d, part);
+    switch (b) {
+        case 4: stage_row<4, true>(xr, C, b, kp, s, d, part); break;
+        case 8: stage_row<8, true>(xr, C, b, kp, s, d, part); break;
+        case 16: stage_row<16, true>(xr, C, b, kp, s, d, part); break;
+        case 32: stage_row<32, true>(xr, C, b, kp, s, d, part); break;
+        default:
+            if (b <= 4) stage_row<4, false>(xr, C, b, kp, s, d, part);
+            else if (b <= 8) stage_row<8, false>(xr, C, b, kp, s, d, part);
+            else if (b <= 16) stage_row<16, false>(xr, C, b, kp, s, d, part);
+            else stage_row<B_MAX, false>(xr, C, b, kp, s, d, part);
+    }
 }
 
 // Lloyd-Max code = number of midpoints t_k below z, found with one table
@@ -251,15 +259,24 @@ __device__ __forceinline__ void quantize_rows(float *xr, const QuantDev &Q, cons
         if (mine && ck < nch) {
             const int q = ck >> lcpg;
             const float s = pick4(sc, q), is = pick4(inv, q);
+            // one of two whole loops, so only one code path is fetched and run
+            if (use_bins && s > 0.0f) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const float x = xr[ck * 32 + e];
-                const unsigned code = static_cast<unsigned>(
-                    (use_bins && s > 0.0f) ? code_binned(x * is, thr, bins)
-                                           : code_of_smem<BITS>(x, s, is, !is_max, thr));
-                const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
-                w[ci][wi] |= code << sh;
-                if (sh + BITS > 32) w[ci][wi + 1] |= code >> (32 - sh);
+                for (int e = 0; e < 32; ++e) {
+                    const unsigned code = static_cast<unsigned>(code_binned(xr[ck * 32 + e] * is, thr, bins));
+                    const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
+                    w[ci][wi] |= code << sh;
+                    if (sh + BITS > 32) w[ci][wi + 1] |= code >> (32 - sh);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const unsigned code = static_cast<unsigned>(
+                        code_of_smem<BITS>(xr[ck * 32 + e], s, is, !is_max, thr));
+                    const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
+                    w[ci][wi] |= code << sh;
+                    if (sh + BITS > 32) w[ci][wi + 1] |= code >> (32 - sh);
+                }
             }
         }
     }
