@@ -54,7 +54,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # DRAM bytes (read + write) per pass launch of this step, from one ncu capture
 # of the current pass kernels (profiles/pass_kernel_c2_4096x4096_traffic.md);
 # writes still in L2 when a launch ends are counted by the next launch.
-MEASURED_TRAFFIC = {"fwd_p0_2bit": 51849216, "fwd_p1_2bit": 88366848, "fwd_p2_2bit": 68218624, "inv_p0_2bit": 17544448, "inv_p1_2bit": 88150016, "inv_p2_2bit": 70254592, "fwd_p0_4bit": 48630272, "fwd_p1_4bit": 87965184, "fwd_p2_4bit": 68028160, "inv_p0_4bit": 21670144, "inv_p1_4bit": 88139520, "inv_p2_4bit": 70288896}
+MEASURED_TRAFFIC = {"fwd_p0_2bit": 51289088, "fwd_p1_2bit": 87449600, "fwd_p2_2bit": 68028416, "inv_p0_2bit": 16413440, "inv_p1_2bit": 87298048, "inv_p2_2bit": 69392640, "fwd_p0_4bit": 48102656, "fwd_p1_4bit": 87410688, "fwd_p2_4bit": 68059904, "inv_p0_4bit": 20436224, "inv_p1_4bit": 87161600, "inv_p2_4bit": 69362688}
 
 
 def fwd_bytes_per_elem(bits):

@@ -2,6 +2,7 @@
 // (harp_kernels.cu). Not installed; the public surface is include/harp.h.
 #pragma once
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 
@@ -50,6 +51,23 @@ struct QuantDev {
     float level[32];  // dequantised level per code (centroid or code - 2^(b-1))
     float thr[32];    // Lloyd-Max midpoints (K - 1 used)
 };
+
+// Whether the binned Lloyd-Max code search (code_binned<nb>: nb bins of
+// width 8/nb over [-4, 4], the edge bins open-ended) is exact for q's fp32
+// midpoints, i.e. no bin holds two of them. Absmax codebooks never use it.
+inline bool bins_exact(const QuantDev &q, int nb) {
+    if (q.kind != HARP_LLOYD_MAX) return false;
+    const int K = 1 << q.bits;
+    int prev = -1;
+    for (int k = 0; k < K - 1; ++k) {
+        // bin i covers [(i - nb/2 - 1/2) * 8/nb, (i - nb/2 + 1/2) * 8/nb)
+        int bin = static_cast<int>(std::floor(static_cast<double>(q.thr[k]) * (nb / 8.0) + nb / 2.0 + 0.5));
+        bin = bin < 0 ? 0 : (bin > nb - 1 ? nb - 1 : bin);
+        if (bin == prev) return false;
+        prev = bin;
+    }
+    return true;
+}
 
 enum Prologue { PRO_F32 = 0, PRO_BF16 = 1, PRO_CODES = 2 };
 enum Epilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_QUANT = 2, EPI_QUANT_F32 = 3, EPI_REQUANT = 4 };

@@ -123,6 +123,7 @@ struct PassDesc {
     int tab_base;       // float offset of the index tables (rows, then cols)
     int smem_bytes;
     int sign_at_store;  // inverse: signs after the stages
+    int bins;           // quantising pass: Lloyd-Max codes by the 64-bin table (exact for these midpoints)
     int in_blocked;     // input is a workspace in this pass's tile-major layout
     int out_blocked;    // output is a workspace in the next pass's tile-major layout
     PAxis nx[2];        // the next pass's tile geometry (out_blocked)
@@ -528,7 +529,8 @@ __device__ __forceinline__ void store_tile(const float *T, const PassDesc &D, co
 // xor tree.
 template <int BITS, bool F32COPY>
 __device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDesc &D, const QuantDev &Q,
-                                                   const Tabs &tb, const float *ts, int warp, int lane) {
+                                                   const Tabs &tb, const float *ts, const unsigned char *bins,
+                                                   int warp, int lane) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     const int g = Q.group, ngt = Ec / g, nit = g >> 5;
     const bool is_max = (Q.kind == HARP_ABSMAX);
@@ -560,10 +562,18 @@ __device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDes
         for (int it = 0; it < nit; ++it) {
             unsigned word = 0;
             float x[8];
+            if (D.bins && s > 0.0f) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                x[e] = rp[32 * it + e];
-                word |= static_cast<unsigned>(code_of_smem<BITS>(x[e], s, inv, !is_max, ts)) << (BITS * e);
+                for (int e = 0; e < 8; ++e) {
+                    x[e] = rp[32 * it + e];
+                    word |= static_cast<unsigned>(code_binned<64>(x[e] * inv, ts, bins)) << (BITS * e);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    x[e] = rp[32 * it + e];
+                    word |= static_cast<unsigned>(code_of_smem<BITS>(x[e], s, inv, !is_max, ts)) << (BITS * e);
+                }
             }
             const int64_t col = c0 + 32 * it + 8 * c;       // first of this lane's 8 columns
             if constexpr (BITS == 4) {
@@ -790,7 +800,10 @@ __device__ __forceinline__ void convert_input(const PassDesc &D, const QuantDev 
 // next tile's input is loaded into registers and its coefficients copied
 // (asynchronously) into the other coefficient buffer before the current
 // tile's stages run, so memory latency overlaps the arithmetic.
-template <int PRO, int EPI>
+// HAD: whether the pass holds a Walsh-Hadamard stage. Passes without one are
+// built without the butterfly code, which otherwise costs the general stages
+// registers and instruction-cache room.
+template <int PRO, int EPI, bool HAD>
 __global__ void __launch_bounds__(PT, 1)
 pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev Q) {
     extern __shared__ float4 sm4[];
@@ -805,7 +818,12 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
     const unsigned ntiles = static_cast<unsigned>(D.ax[0].nt * D.ax[1].nt);
     unsigned t = blockIdx.x;
     if (t >= ntiles) return;
-    if (tid < 16) {
+    if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
+        // a quantising pass decodes nothing: the level slots hold the bin table
+        const int K = 1 << Q.bits;
+        if (tid < 16) lev[16 + tid] = (tid < K - 1) ? Q.thr[tid] : __int_as_float(0x7f800000);
+        if (D.bins && tid < 64) reinterpret_cast<unsigned char *>(lev)[tid] = bin_entry<64>(tid, Q.thr, K);
+    } else if (tid < 16) {
         lev[tid] = Q.level[tid];
         lev[16 + tid] = Q.thr[tid];     // midpoints (Lloyd-Max code search)
     }
@@ -848,7 +866,7 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
             const PStage &S = D.st[u];
             const bool rows = (S.axis == 0);
             const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
-            if (S.had) {
+            if (HAD && S.had) {
                 switch (S.b) {
                     case 2: stage_fwht<2>(T, S, A, Bv, NV, warp, lane); break;
                     case 4: stage_fwht<4>(T, S, A, Bv, NV, warp, lane); break;
@@ -864,8 +882,9 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
 
         if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
             constexpr bool F = (EPI == EPI_QUANT_F32);
-            if (Q.bits == 2) quantize_tile_fast<2, F>(T, D, Q, B.tb, lev + 16, warp, lane);
-            else if (Q.bits == 4) quantize_tile_fast<4, F>(T, D, Q, B.tb, lev + 16, warp, lane);
+            const unsigned char *bins = reinterpret_cast<const unsigned char *>(lev);
+            if (Q.bits == 2) quantize_tile_fast<2, F>(T, D, Q, B.tb, lev + 16, bins, warp, lane);
+            else if (Q.bits == 4) quantize_tile_fast<4, F>(T, D, Q, B.tb, lev + 16, bins, warp, lane);
             else quantize_tile<3, F>(T, D, Q, B.tb, warp, lane);
         } else {
             store_tile<EPI>(T, D, B.tb, D.sign_at_store && has_sign, warp, lane);
@@ -1141,15 +1160,15 @@ void fill_stages(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inve
     }
 }
 
-template <int PRO, int EPI>
-int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
+template <int PRO, int EPI, bool HAD>
+int launch_pass_t(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     static int attr_done[64] = {};
     static int nsm[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(pass_kernel<PRO, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(pass_kernel<PRO, EPI, HAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              SMEM_BUDGET);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&nsm[dev], cudaDevAttrMultiProcessorCount, dev);
@@ -1159,8 +1178,15 @@ int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     const int64_t nb = D.ax[0].nt * D.ax[1].nt;
     if (nb <= 0) return 0;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(nb, nsm[dev]));
-    pass_kernel<PRO, EPI><<<grid, PT, D.smem_bytes, st>>>(D, Q);
+    pass_kernel<PRO, EPI, HAD><<<grid, PT, D.smem_bytes, st>>>(D, Q);
     return cudaGetLastError();
+}
+
+template <int PRO, int EPI>
+int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
+    bool had = false;
+    for (int u = 0; u < D.nst; ++u) had = had || D.st[u].had;
+    return had ? launch_pass_t<PRO, EPI, true>(D, Q, st) : launch_pass_t<PRO, EPI, false>(D, Q, st);
 }
 
 int dispatch(const PassDesc &D, const QuantDev &Q, int pro, int epi, cudaStream_t st) {
@@ -1296,6 +1322,7 @@ int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q
         if (first) pro = (in_dtype == HARP_BF16) ? PRO_BF16 : PRO_F32;
         if (last) {
             epi = rotated_out ? EPI_QUANT_F32 : EPI_QUANT;
+            D.bins = bins_exact(q, 64) ? 1 : 0;
             D.codes = codes;
             D.scales = scales;
             D.out_f32 = rotated_out;

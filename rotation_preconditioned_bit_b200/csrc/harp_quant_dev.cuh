@@ -92,6 +92,32 @@ __device__ __forceinline__ int code_of_smem(float x, float s, float inv_s, bool 
     return static_cast<int>(fminf(fmaxf(rintf(z), -qmax), qmax)) + HALF;
 }
 
+// Lloyd-Max code = number of midpoints below z by one table read and one
+// compare: NB bins of width 8/NB over [-4, 4]; bin = rint(z * NB/8 + NB/2)
+// clamped to [0, NB - 1] (one rounding of an exact product-sum, so z lies in
+// [(bin - NB/2 - 1/2) * 8/NB, (bin - NB/2 + 1/2) * 8/NB] unless clamped);
+// bins[bin] = number of midpoints below that lower edge (0 for bin 0). Exact
+// when no bin holds two midpoints (bins_exact on the host); thr[K - 1] must
+// be +inf.
+template <int NB>
+__device__ __forceinline__ int code_binned(float z, const float *thr, const unsigned char *bins) {
+    const float y = fmaf(z, static_cast<float>(NB / 8), static_cast<float>(NB / 2) + 12582912.0f);  // 1.5 * 2^23
+    int bin = __float_as_int(y) - 0x4B400000;
+    bin = min(max(bin, 0), NB - 1);
+    const int c = bins[bin];
+    return c + ((z > thr[c]) ? 1 : 0);
+}
+
+// Entry i of that table, for thread i < NB (K - 1 midpoints in thr).
+template <int NB>
+__device__ __forceinline__ unsigned char bin_entry(int i, const float *thr, int K) {
+    if (i == 0) return 0;
+    const float lo = (static_cast<float>(i - NB / 2) - 0.5f) * (8.0f / NB);
+    int c = 0;
+    for (int k = 0; k < K - 1; ++k) c += (thr[k] < lo) ? 1 : 0;
+    return static_cast<unsigned char>(c);
+}
+
 template <int BITS>
 __device__ __forceinline__ unsigned pack_words(int code, int lane) {
     const int bit0 = BITS * lane;

@@ -185,21 +185,6 @@ __device__ __forceinline__ void run_stage_row(float *xr, const float *C, const S
     }
 }
 
-// Lloyd-Max code = number of midpoints t_k below z, found with one table
-// read and one compare: bin = rint(32 z + 128) clamped to [0, 255] (a single
-// rounding of an exact product-sum: z lies in [(bin - 128.5)/32,
-// (bin - 127.5)/32] unless clamped), bins[bin] = number of midpoints below
-// the bin's lower edge (0 for bin 0), and the host has checked that no bin
-// holds two midpoints (the edge bins included, open-ended), so the code is
-// bins[bin] or one more. thr[K - 1] is +inf.
-__device__ __forceinline__ int code_binned(float z, const float *thr, const unsigned char *bins) {
-    const float y = fmaf(z, 32.0f, 128.0f + 12582912.0f);     // 12582912 = 1.5 * 2^23
-    int bin = __float_as_int(y) - 0x4B400000;
-    bin = min(max(bin, 0), 255);
-    const int c = bins[bin];
-    return c + ((z > thr[c]) ? 1 : 0);
-}
-
 // One of the 4 values a[0..3] picked by a runtime index (registers only).
 __device__ __forceinline__ float pick4(const float (&a)[4], int i) {
     return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
@@ -263,7 +248,7 @@ __device__ __forceinline__ void quantize_rows(float *xr, const QuantDev &Q, cons
             if (use_bins && s > 0.0f) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const unsigned code = static_cast<unsigned>(code_binned(xr[ck * 32 + e] * is, thr, bins));
+                    const unsigned code = static_cast<unsigned>(code_binned<256>(xr[ck * 32 + e] * is, thr, bins));
                     const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
                     w[ci][wi] |= code << sh;
                     if (sh + BITS > 32) w[ci][wi + 1] |= code >> (32 - sh);
@@ -365,14 +350,7 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             lev[tid] = Q.level[tid];
             thr[tid] = (tid < K - 1) ? QO.thr[tid] : __int_as_float(0x7f800000);
         }
-        if (L.bins && tid < 256) {
-            // bins[i] = number of midpoints below (i - 128.5) / 32; bin 0 open below
-            const float lo = (static_cast<float>(tid) - 128.5f) * 0.03125f;
-            int c = 0;
-            if (tid > 0)
-                for (int k = 0; k < K - 1; ++k) c += (QO.thr[k] < lo) ? 1 : 0;
-            bins[tid] = static_cast<unsigned char>(c);
-        }
+        if (L.bins && tid < 256) bins[tid] = bin_entry<256>(tid, QO.thr, K);
     }
 
     const int64_t ntiles = (L.nvec + ST - 1) / ST;
@@ -524,27 +502,10 @@ bool short_ok(const PlanDev &P, int mode, int in_bits) {
     return short_smem_bytes(P, mode, in_bits) <= SMEM_LIMIT;
 }
 
-// Whether the bin table of code_binned is exact for these midpoints: no bin
-// [(i - 128.5)/32, (i - 127.5)/32) (bin 0 open below, bin 255 open above)
-// holds two of them.
-bool bins_exact(const QuantDev &q) {
-    if (q.kind != HARP_LLOYD_MAX) return false;
-    const int K = 1 << q.bits;
-    int prev_bin = -1;
-    for (int k = 0; k < K - 1; ++k) {
-        const double t = static_cast<double>(q.thr[k]);
-        int bin = static_cast<int>(std::floor((t * 32.0 + 128.5)));   // t in [lo_bin, lo_bin + 1/32)
-        bin = bin < 0 ? 0 : (bin > 255 ? 255 : bin);
-        if (bin == prev_bin) return false;
-        prev_bin = bin;
-    }
-    return true;
-}
-
 int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &Lin, void *stream) {
     if (Lin.nvec == 0) return cudaSuccess;
     ShortLaunch L = Lin;
-    L.bins = (L.mode == SHORT_INV) ? 0 : (bins_exact(L.mode == SHORT_REQUANT ? L.q2 : q) ? 1 : 0);
+    L.bins = (L.mode == SHORT_INV) ? 0 : (bins_exact(L.mode == SHORT_REQUANT ? L.q2 : q, 256) ? 1 : 0);
     const int in_bits = (L.mode == SHORT_FWD) ? 0 : q.bits;
     const size_t smem = short_smem_bytes(P, L.mode, in_bits);
     const void *fn = (L.mode == SHORT_FWD) ? reinterpret_cast<const void *>(short_kernel<SHORT_FWD>)
