@@ -800,10 +800,16 @@ __device__ __forceinline__ void convert_input(const PassDesc &D, const QuantDev 
 // next tile's input is loaded into registers and its coefficients copied
 // (asynchronously) into the other coefficient buffer before the current
 // tile's stages run, so memory latency overlaps the arithmetic.
-// HAD: whether the pass holds a Walsh-Hadamard stage. Passes without one are
-// built without the butterfly code, which otherwise costs the general stages
-// registers and instruction-cache room.
-template <int PRO, int EPI, bool HAD>
+// Stage paths a build carries: every pass kernel is built three times, so a
+// pass runs the build with only the stage code it needs (unused paths cost
+// the others registers and instruction-cache room).
+enum StageSet {
+    SS_ALL = 0,    // Walsh-Hadamard butterflies and all block widths
+    SS_BLOCKS = 1, // block stages of any width, no butterfly
+    SS_K16 = 2     // only block stages of 9..16 outputs (kp = 16)
+};
+
+template <int PRO, int EPI, int SS>
 __global__ void __launch_bounds__(PT, 1)
 pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev Q) {
     extern __shared__ float4 sm4[];
@@ -866,17 +872,21 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
             const PStage &S = D.st[u];
             const bool rows = (S.axis == 0);
             const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
-            if (HAD && S.had) {
-                switch (S.b) {
-                    case 2: stage_fwht<2>(T, S, A, Bv, NV, warp, lane); break;
-                    case 4: stage_fwht<4>(T, S, A, Bv, NV, warp, lane); break;
-                    case 8: stage_fwht<8>(T, S, A, Bv, NV, warp, lane); break;
-                    case 16: stage_fwht<16>(T, S, A, Bv, NV, warp, lane); break;
-                    default: stage_fwht<32>(T, S, A, Bv, NV, warp, lane); break;
-                }
-            } else if (S.kp == 8) stage_run<8, false>(T, B.C, S, A, Bv, NV, warp, lane);
-            else if (S.kp == 16) stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
-            else stage_rounds(T, B.C, S, A, Bv, NV, warp, lane);
+            if constexpr (SS == SS_K16) {
+                stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
+            } else {
+                if (SS == SS_ALL && S.had) {
+                    switch (S.b) {
+                        case 2: stage_fwht<2>(T, S, A, Bv, NV, warp, lane); break;
+                        case 4: stage_fwht<4>(T, S, A, Bv, NV, warp, lane); break;
+                        case 8: stage_fwht<8>(T, S, A, Bv, NV, warp, lane); break;
+                        case 16: stage_fwht<16>(T, S, A, Bv, NV, warp, lane); break;
+                        default: stage_fwht<32>(T, S, A, Bv, NV, warp, lane); break;
+                    }
+                } else if (S.kp == 8) stage_run<8, false>(T, B.C, S, A, Bv, NV, warp, lane);
+                else if (S.kp == 16) stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
+                else stage_rounds(T, B.C, S, A, Bv, NV, warp, lane);
+            }
             __syncthreads();
         }
 
@@ -1160,7 +1170,7 @@ void fill_stages(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inve
     }
 }
 
-template <int PRO, int EPI, bool HAD>
+template <int PRO, int EPI, int SS>
 int launch_pass_t(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     static int attr_done[64] = {};
     static int nsm[64] = {};
@@ -1168,7 +1178,7 @@ int launch_pass_t(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(pass_kernel<PRO, EPI, HAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(pass_kernel<PRO, EPI, SS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              SMEM_BUDGET);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&nsm[dev], cudaDevAttrMultiProcessorCount, dev);
@@ -1178,15 +1188,20 @@ int launch_pass_t(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     const int64_t nb = D.ax[0].nt * D.ax[1].nt;
     if (nb <= 0) return 0;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(nb, nsm[dev]));
-    pass_kernel<PRO, EPI, HAD><<<grid, PT, D.smem_bytes, st>>>(D, Q);
+    pass_kernel<PRO, EPI, SS><<<grid, PT, D.smem_bytes, st>>>(D, Q);
     return cudaGetLastError();
 }
 
 template <int PRO, int EPI>
 int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
-    bool had = false;
-    for (int u = 0; u < D.nst; ++u) had = had || D.st[u].had;
-    return had ? launch_pass_t<PRO, EPI, true>(D, Q, st) : launch_pass_t<PRO, EPI, false>(D, Q, st);
+    bool had = false, k16 = true;
+    for (int u = 0; u < D.nst; ++u) {
+        had = had || D.st[u].had;
+        k16 = k16 && !D.st[u].had && D.st[u].kp == 16 && D.st[u].b <= 16;
+    }
+    if (had) return launch_pass_t<PRO, EPI, SS_ALL>(D, Q, st);
+    if (k16) return launch_pass_t<PRO, EPI, SS_K16>(D, Q, st);
+    return launch_pass_t<PRO, EPI, SS_BLOCKS>(D, Q, st);
 }
 
 int dispatch(const PassDesc &D, const QuantDev &Q, int pro, int epi, cudaStream_t st) {
