@@ -180,8 +180,9 @@ int harp_theta_blocks(int b, int64_t n_groups, const int8_t *theta, float theta_
  * ones the new; launches on other streams must be ordered by the caller. The
  * stage is afterwards applied by general block arithmetic (never the
  * Walsh-Hadamard butterfly), also when every q is 0.
+ * Must be called with the plan's device current.
  * Errors: INVALID_ARG (NULL plan or pointer, stage outside [0, m), non-finite
- * scale, missing base), CUDA. */
+ * scale, missing base, another device current), CUDA. */
 int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float theta_scale,
                          const float *base, void *stream);
 

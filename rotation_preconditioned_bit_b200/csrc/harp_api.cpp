@@ -396,6 +396,9 @@ int harp_theta_blocks(int b, int64_t n_groups, const int8_t *theta, float theta_
 int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float theta_scale,
                          const float *base, void *stream) {
     if (!plan || stage < 0 || stage >= plan->m) return HARP_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HARP_ERR_CUDA; }
+    if (dev != plan->device) return HARP_ERR_INVALID_ARG;   // the plan's memory lives on its own device
     harp::StageDev &sd = plan->dev.st[stage];
     const int b = sd.b;
     const int64_t ng = plan->d / b;
