@@ -234,9 +234,12 @@ __device__ __forceinline__ void unit_addr(const PStage &S, int gi, int v0, int L
 // w[j][0..K) is read as K/4 16-byte words, each two ready-made pairs, and
 // x_v[j] is broadcast into both halves. CLAMP: inputs past b are read at b-1
 // and meet zero coefficients (only when b is not a multiple of 4).
-template <int K, bool CLAMP>
-__device__ __forceinline__ void unit_compute(const float *T, const float *wp, int kp, int jpad, int b,
+// EXACT: b = jpad = kp = K (fixed trip count, no clamping): the loop is
+// unrolled completely.
+template <int K, bool CLAMP, bool EXACT = false>
+__device__ __forceinline__ void unit_compute(const float *T, const float *wp, int kp_rt, int jpad_rt, int b_rt,
                                              int step, const int (&p)[VL], f2_t (&acc)[K / 2][VL]) {
+    const int kp = EXACT ? K : kp_rt, jpad = EXACT ? K : jpad_rt, b = EXACT ? K : b_rt;
 #pragma unroll
     for (int q = 0; q < K / 2; ++q)
 #pragma unroll
@@ -247,7 +250,7 @@ __device__ __forceinline__ void unit_compute(const float *T, const float *wp, in
     const ulonglong2 *wq = reinterpret_cast<const ulonglong2 *>(wp);
     const int wstep = kp / 4;      // 16-byte words per coefficient row
     const int jlast = (b - 1) * step;
-#pragma unroll 4
+#pragma unroll(EXACT ? K : 4)
     for (int j = 0; j < jpad; ++j) {
         f2_t x[VL];
 #pragma unroll
@@ -294,7 +297,8 @@ __device__ __forceinline__ void unit_store(float *T, int b, int k0, int step, co
 // without barriers. Wider blocks (ROUNDS) split the outputs into chunks of K
 // over several warps, which first all read (compute into registers), then
 // all write; the warps of one round hold whole (group block, vector block)s.
-template <int K, bool ROUNDS>
+// EXACT (no ROUNDS): every block of the stage has b = K outputs and inputs.
+template <int K, bool ROUNDS, bool EXACT = false>
 __device__ __forceinline__ void stage_run(float *T, const float *C, const PStage &S, int A, int Bv, int NV,
                                           int warp, int lane) {
     const int LV = S.LV, LG = 32 / LV;
@@ -315,9 +319,14 @@ __device__ __forceinline__ void stage_run(float *T, const float *C, const PStage
             const float *wp;
             unit_addr(S, gb * LG + lg, vc * span + lv, LV, NV, A, Bv, Cs, p, vok, gok, wp);
             f2_t acc[K / 2][VL];
-            if (clamp) unit_compute<K, true>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
-            else unit_compute<K, false>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
-            unit_store<K>(T, S.b, 0, step, p, vok, gok, acc);
+            if constexpr (EXACT) {
+                unit_compute<K, false, true>(T, wp, K, K, K, step, p, acc);
+                unit_store<K>(T, K, 0, step, p, vok, gok, acc);
+            } else {
+                if (clamp) unit_compute<K, true>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
+                else unit_compute<K, false>(T, wp, S.kp, S.jpad, S.b, step, p, acc);
+                unit_store<K>(T, S.b, 0, step, p, vok, gok, acc);
+            }
         }
     } else {
         const int nblk = ngb * nvc;
@@ -806,7 +815,7 @@ __device__ __forceinline__ void convert_input(const PassDesc &D, const QuantDev 
 enum StageSet {
     SS_ALL = 0,    // Walsh-Hadamard butterflies and all block widths
     SS_BLOCKS = 1, // block stages of any width, no butterfly
-    SS_K16 = 2     // only block stages of 9..16 outputs (kp = 16)
+    SS_K16 = 2     // only block stages of exactly 16 outputs and inputs
 };
 
 template <int PRO, int EPI, int SS>
@@ -873,7 +882,7 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
             const bool rows = (S.axis == 0);
             const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
             if constexpr (SS == SS_K16) {
-                stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
+                stage_run<16, false, true>(T, B.C, S, A, Bv, NV, warp, lane);
             } else {
                 if (SS == SS_ALL && S.had) {
                     switch (S.b) {
@@ -1197,7 +1206,7 @@ int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     bool had = false, k16 = true;
     for (int u = 0; u < D.nst; ++u) {
         had = had || D.st[u].had;
-        k16 = k16 && !D.st[u].had && D.st[u].kp == 16 && D.st[u].b <= 16;
+        k16 = k16 && !D.st[u].had && D.st[u].b == 16 && D.st[u].kp == 16 && D.st[u].jpad == 16;
     }
     if (had) return launch_pass_t<PRO, EPI, SS_ALL>(D, Q, st);
     if (k16) return launch_pass_t<PRO, EPI, SS_K16>(D, Q, st);
