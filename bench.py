@@ -54,7 +54,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # DRAM bytes (read + write) per pass launch of this step, from one ncu capture
 # of the current pass kernels (profiles/pass_kernel_c2_4096x4096_traffic.md);
 # writes still in L2 when a launch ends are counted by the next launch.
-MEASURED_TRAFFIC = {"fwd_p0_2bit": 50286080, "fwd_p1_2bit": 86665472, "fwd_p2_2bit": 67989248, "inv_p0_2bit": 16491520, "inv_p1_2bit": 87004928, "inv_p2_2bit": 69238272, "fwd_p0_4bit": 47579392, "fwd_p1_4bit": 87122176, "fwd_p2_4bit": 68087808, "inv_p0_4bit": 20798208, "inv_p1_4bit": 86690816, "inv_p2_4bit": 69271808}
+MEASURED_TRAFFIC = {"fwd_p0_2bit": 50772992, "fwd_p1_2bit": 87244800, "fwd_p2_2bit": 67990016, "inv_p0_2bit": 16310272, "inv_p1_2bit": 86892800, "inv_p2_2bit": 69811968, "fwd_p0_4bit": 47464704, "fwd_p1_4bit": 87061760, "fwd_p2_4bit": 67991808, "inv_p0_4bit": 20769024, "inv_p1_4bit": 86921472, "inv_p2_4bit": 69498112}
 
 
 def fwd_bytes_per_elem(bits):
