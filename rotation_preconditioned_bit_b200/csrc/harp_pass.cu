@@ -893,6 +893,8 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
                         default: stage_fwht<32>(T, S, A, Bv, NV, warp, lane); break;
                     }
                 } else if (S.kp == 8) stage_run<8, false>(T, B.C, S, A, Bv, NV, warp, lane);
+                else if (S.kp == 16 && S.b == 16 && S.jpad == 16)
+                    stage_run<16, false, true>(T, B.C, S, A, Bv, NV, warp, lane);
                 else if (S.kp == 16) stage_run<16, false>(T, B.C, S, A, Bv, NV, warp, lane);
                 else stage_rounds(T, B.C, S, A, Bv, NV, warp, lane);
             }
