@@ -51,10 +51,26 @@ WORKLOAD = ("4096x4096 bf16 weight (Student-t nu=3 x0.02, 0.5% input channels x2
             "dequantize+unrotate for each bit width")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 
-# DRAM bytes (read + write) per pass launch of this step, from one ncu capture
-# of the current pass kernels (profiles/pass_kernel_c2_4096x4096_traffic.md);
-# writes still in L2 when a launch ends are counted by the next launch.
-MEASURED_TRAFFIC = {"fwd_p0_2bit": 50772992, "fwd_p1_2bit": 87244800, "fwd_p2_2bit": 67990016, "inv_p0_2bit": 16310272, "inv_p1_2bit": 86892800, "inv_p2_2bit": 69811968, "fwd_p0_4bit": 47464704, "fwd_p1_4bit": 87061760, "fwd_p2_4bit": 67991808, "inv_p0_4bit": 20769024, "inv_p1_4bit": 86921472, "inv_p2_4bit": 69498112}
+# DRAM bytes (read + write) per pass launch of this step, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the pass kernels
+# built from the source whose SHA-256 prefix is "kernel_src"; writes still in
+# L2 when a launch ends are counted by the next launch. When the pass-kernel
+# source differs from the captured one the figures no longer describe the
+# kernel and the roofline's traffic field is reported as null.
+MEASURED_TRAFFIC = {"kernel_src": None, "bytes": {}}
+PASS_SRC = os.path.join(ROOT, "rotation_preconditioned_bit_b200", "csrc", "harp_pass.cu")
+
+
+def pass_source_hash():
+    import hashlib
+    with open(PASS_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(kernel):
+    if MEASURED_TRAFFIC["kernel_src"] != pass_source_hash():
+        return None
+    return MEASURED_TRAFFIC["bytes"].get(kernel)
 
 
 def fwd_bytes_per_elem(bits):
@@ -617,7 +633,7 @@ def main():
         d = ktab[dom]
         roof = {"kernel": dom, "bound": "alu", "achieved": d["tflops"], "peak": round(peak_tf, 1),
                 "unit": "TFLOP/s", "frac": round(d["tflops"] / peak_tf, 4),
-                "traffic": MEASURED_TRAFFIC.get(dom),
+                "traffic": measured_traffic(dom),
                 "peak_source": f"FFMA: 148 SM x 128 lanes x 2 flop x {smhz:.0f} MHz (max SM clock, {peak_src})",
                 "algorithmic": f"2 flop per block coefficient per element: FMA per element by forward pass {pass_fma}",
                 "own_bytes_hbm_frac": round(d["own_gbs"] / hbm, 4)}

@@ -317,6 +317,34 @@ int harp_pass_fma(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int p
  * INVALID_ARG (n < 0, or NULL events with n > 0). */
 int harp_set_pass_events(void *const *events, int n);
 
+/* ------------------------------------------------------------ diagnostics */
+
+/* Which arithmetic the two-sided calls' block stages use (process-wide; a
+ * tuning and testing switch, results agree within the fp32 tolerance):
+ *  HARP_BLOCK_STAGES_AUTO  per pass, tensor cores (tcgen05.mma kind::tf32
+ *                          with split operands, "3xTF32": each product
+ *                          x*b as x_hi*b_hi + x_lo*b_hi + x_hi*b_lo in fp32)
+ *                          when a block of the pass is wider than 32, else
+ *                          fp32 FMAs (the faster of the two measured on the
+ *                          B200 for each width);
+ *  HARP_BLOCK_STAGES_TC    tensor cores for every block stage;
+ *  HARP_BLOCK_STAGES_FFMA  fp32 FMAs for every block stage.
+ * Stages whose blocks are all normalised Sylvester matrices always run as
+ * Walsh-Hadamard butterflies. Takes effect for calls made afterwards.
+ * Errors: INVALID_ARG (unknown mode). */
+enum harp_block_stages { HARP_BLOCK_STAGES_AUTO = 0, HARP_BLOCK_STAGES_TC = 1, HARP_BLOCK_STAGES_FFMA = 2 };
+int harp_set_block_stages(int mode);
+
+/* Every wait inside the library's kernels is bounded (the tensor-core stages
+ * of the two-sided kernels wait for their MMA batches for about half a
+ * second at most); a wait that runs out abandons the launch without trapping
+ * and is recorded per device. This call returns that record for the current
+ * device in *flags and clears it: 0 = no wait ran out; bit 0 = a tensor-core
+ * batch of a two-sided call did not complete (that call's outputs are
+ * incomplete). Synchronous (it waits for the device's pending work).
+ * Errors: INVALID_ARG (NULL flags), CUDA. */
+int harp_fault_status(unsigned int *flags);
+
 /* ------------------------------------------- variant that allocates nothing */
 
 /* Capacity of the library-owned scratch used by harp_rotate_quantize_static:

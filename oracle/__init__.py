@@ -29,9 +29,10 @@ BLOCK_KINDS = {"hadamard": 0, "qr": 1, "cayley_hadamard": 2}
 
 
 def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so (gcc, -O2, no fast-math)."""
+    """Compile oracle.c into liboracle.so (gcc, -O2, no fast-math; OpenMP
+    spreads its independent rows / columns over the host threads)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-D_DEFAULT_SOURCE", "-fPIC",
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-D_DEFAULT_SOURCE", "-fPIC", "-fopenmp",
                                "-shared", "-o", _LIB, _SRC, "-lm"])
     return _LIB
 
@@ -80,8 +81,16 @@ def _set_types(L):
     L.orc_dequantize.argtypes = [_INT, _INT, _L, _L, _L, _U8, _U16, _D]
     L.orc_pack.argtypes = [_INT, _L, _L, _U8, _U8]
     L.orc_unpack.argtypes = [_INT, _L, _L, _U8, _U8]
+    L.orc_threads.argtypes = [_INT]
+    L.orc_threads.restype = _INT
     L.orc_two_sided_rows.argtypes = [_L, _L, _INT, _I32, _D, _D, _INT, _I32, _D, _D, _D, _L, _I64, _D]
     L.orc_inverse_rows.argtypes = [_L, _L, _INT, _I32, _D, _D, _INT, _I32, _D, _D, _D, _L, _I64, _D]
+
+
+def threads(n: int = 0) -> int:
+    """Set the number of host threads of the oracle's row / column loops
+    (n <= 0: unchanged); returns the current number."""
+    return int(lib().orc_threads(int(n)))
 
 
 def _p(a, t):

@@ -41,6 +41,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_BAD 1
@@ -122,35 +125,68 @@ int orc_apply(int64_t d, int m, const int32_t *radix, const double *blocks,
     return ORC_OK;
 }
 
-/* Right side: every row r of X [rows x cols] becomes M r  (X -> X M^T). */
+/* Right side: every row r of X [rows x cols] becomes M r  (X -> X M^T).
+ * Rows are independent; with OpenMP they are spread over the host threads
+ * (the arithmetic of each row is unchanged). */
 int orc_rotate_rows(int64_t rows, int64_t cols, int m, const int32_t *radix,
                     const double *blocks, const double *signs, int inverse,
                     const double *X, double *Y)
 {
+    int st = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 16)
     for (int64_t r = 0; r < rows; ++r) {
-        int st = orc_apply(cols, m, radix, blocks, signs, inverse, X + r * cols, Y + r * cols);
-        if (st) return st;
+        if (orc_apply(cols, m, radix, blocks, signs, inverse, X + r * cols, Y + r * cols)) {
+#pragma omp atomic write
+            st = ORC_BAD;
+        }
     }
-    return ORC_OK;
+    return st;
 }
 
-/* Left side: every column w of X [rows x cols] becomes M w  (X -> M X). */
+/* Left side: every column w of X [rows x cols] becomes M w  (X -> M X).
+ * Columns are independent (OpenMP over columns, one gather buffer per
+ * thread). */
 int orc_rotate_cols(int64_t rows, int64_t cols, int m, const int32_t *radix,
                     const double *blocks, const double *signs, int inverse,
                     const double *X, double *Y)
 {
-    double *u = (double *)malloc(sizeof(double) * rows);
-    double *v = (double *)malloc(sizeof(double) * rows);
-    if (!u || !v) { free(u); free(v); return ORC_BAD; }
-    for (int64_t c = 0; c < cols; ++c) {
-        for (int64_t r = 0; r < rows; ++r) u[r] = X[r * cols + c];
-        int st = orc_apply(rows, m, radix, blocks, signs, inverse, u, v);
-        if (st) { free(u); free(v); return st; }
-        for (int64_t r = 0; r < rows; ++r) Y[r * cols + c] = v[r];
+    int st = ORC_OK;
+#pragma omp parallel
+    {
+        double *u = (double *)malloc(sizeof(double) * rows);
+        double *v = (double *)malloc(sizeof(double) * rows);
+        if (!u || !v) {
+#pragma omp atomic write
+            st = ORC_BAD;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t c = 0; c < cols; ++c) {
+            if (!u || !v) continue;
+            for (int64_t r = 0; r < rows; ++r) u[r] = X[r * cols + c];
+            if (orc_apply(rows, m, radix, blocks, signs, inverse, u, v)) {
+#pragma omp atomic write
+                st = ORC_BAD;
+                continue;
+            }
+            for (int64_t r = 0; r < rows; ++r) Y[r * cols + c] = v[r];
+        }
+        free(u);
+        free(v);
     }
-    free(u);
-    free(v);
-    return ORC_OK;
+    return st;
+}
+
+/* Host threads the oracle's row / column loops use (OpenMP); n <= 0 leaves
+ * the setting unchanged. Returns the current maximum. */
+int orc_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
 }
 
 /* Dense stage matrices for tiny d: S_t[i][i'] = B[t][c][k][j] where
@@ -552,6 +588,7 @@ int orc_quantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
         orc_tables(bits, c64, cent, thr);
     }
     int64_t ng = cols / group;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t g = 0; g < ng; ++g) {
             const double *x = X + r * cols + g * group;
@@ -652,6 +689,7 @@ int orc_dequantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols
         orc_tables(bits, c64, cent, thr);
     }
     int64_t ng = cols / group;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t i = 0; i < cols; ++i) {
             double s = orc_f16_value(scales[r * ng + i / group]);

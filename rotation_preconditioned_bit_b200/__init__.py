@@ -40,7 +40,8 @@ EXPORTS = (
     "harp_workspace_size", "harp_rotate", "harp_quantize", "harp_dequantize",
     "harp_rotate_quantize", "harp_dequantize_unrotate", "harp_rotate_quantize_static",
     "harp_pass_count", "harp_pass_fma", "harp_set_pass_events",
-    "harp_theta_blocks", "harp_plan_load_theta", "harp_requantize",
+    "harp_theta_blocks", "harp_plan_load_theta", "harp_requantize", "harp_fault_status",
+    "harp_set_block_stages",
 )
 
 
@@ -91,6 +92,8 @@ def lib():
         L.harp_theta_blocks.argtypes = [_INT, _I64, _P, ctypes.c_float, _P, _P, _P]
         L.harp_plan_load_theta.argtypes = [_P, _INT, _P, ctypes.c_float, _P, _P]
         L.harp_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _INT, _P, _P, _P, _P, _P]
+        L.harp_fault_status.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.harp_set_block_stages.argtypes = [_INT]
         _lib = L
     return _lib
 
@@ -287,6 +290,23 @@ def harp_pass_fma(left, right, cb, k) -> int:
     n = ctypes.c_int()
     _check(lib().harp_pass_fma(left.handle, right.handle, cb.handle, k, ctypes.byref(n)), "harp_pass_fma")
     return n.value
+
+
+HARP_BLOCK_STAGES_AUTO, HARP_BLOCK_STAGES_TC, HARP_BLOCK_STAGES_FFMA = 0, 1, 2
+
+
+def harp_set_block_stages(mode: int) -> None:
+    """Block-stage arithmetic of the two-sided calls: HARP_BLOCK_STAGES_AUTO
+    (per pass, the faster of the two), _TC (tensor cores, 3xTF32) or _FFMA."""
+    _check(lib().harp_set_block_stages(int(mode)), "harp_set_block_stages")
+
+
+def harp_fault_status() -> int:
+    """The current device's record of bounded kernel waits that ran out
+    (0 = none), cleared by the read. Synchronises the device."""
+    v = ctypes.c_uint(0)
+    _check(lib().harp_fault_status(ctypes.byref(v)), "harp_fault_status")
+    return int(v.value)
 
 
 _event_array = None

@@ -54,6 +54,18 @@ bool all_sylvester(int b, int64_t n_groups, const float *B) {
 // Padded block shape of the pass kernels (see StageDev).
 int pass_jpad(int b) { return (b + 3) & ~3; }
 int pass_kp(int b) { return b <= 8 ? 8 : (b + 15) & ~15; }
+int umma_up(int b) { return (b + 15) & ~15; }
+
+// tf32 rounding as tcgen05's tf32 operands see it (10 stored mantissa bits):
+// round to nearest, ties away from zero, on the 13 dropped bits.
+float tf32_rna(float x) {
+    uint32_t u;
+    std::memcpy(&u, &x, 4);
+    if ((u & 0x7f800000u) != 0x7f800000u) u = (u + 0x1000u) & 0xffffe000u;
+    float r;
+    std::memcpy(&r, &u, 4);
+    return r;
+}
 
 // ------------------------------------------------------------ block makers
 // HARP (gist.science paper 2605.29843) section 2.2: B = Q(theta) G_b.
@@ -193,6 +205,19 @@ int theta_args_ok(int b, int64_t n_groups, const int8_t *theta, float theta_scal
 
 // ================================================================ C ABI
 
+namespace harp {
+
+int plans_on_current_device(harp_plan_t a, harp_plan_t b) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HARP_ERR_CUDA; }
+    if ((a && a->device != dev) || (b && b->device != dev)) return HARP_ERR_INVALID_ARG;
+    return HARP_OK;
+}
+
+}  // namespace harp
+
+using harp::plans_on_current_device;
+
 extern "C" {
 
 const char *harp_status_string(int status) {
@@ -295,7 +320,7 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
     // host staging of the device layout
     const size_t sign_floats = (static_cast<size_t>(d) + 3) & ~static_cast<size_t>(3);
     size_t total = sign_floats;
-    std::vector<size_t> off(m), poff(m);
+    std::vector<size_t> off(m), poff(m), uoff(m);
     for (int t = 0; t < m; ++t) {
         const int kpad = (radix[t] + 3) & ~3;
         off[t] = total;
@@ -305,6 +330,11 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
         const int b = radix[t];
         poff[t] = total;
         total += 2 * static_cast<size_t>(d / b) * pass_jpad(b) * pass_kp(b);
+    }
+    for (int t = 0; t < m; ++t) {                       // tensor-core operand layout
+        const int up = umma_up(radix[t]);
+        uoff[t] = total;
+        total += 2 * static_cast<size_t>(d / radix[t]) * 2 * up * up;
     }
     std::vector<float> host;
     try { host.assign(total, 0.0f); } catch (...) { return HARP_ERR_ALLOC; }
@@ -331,6 +361,22 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
                 for (int k = 0; k < b; ++k) {
                     pf[(c * jp + j) * kp + k] = B[k * b + j];
                     pi[(c * jp + j) * kp + k] = B[j * b + k];
+                }
+        }
+        const int up = umma_up(b);
+        const size_t ublk = static_cast<size_t>(2) * up * up;
+        float *uf = host.data() + uoff[t];
+        float *ui = uf + static_cast<size_t>(ng) * ublk;
+        for (int64_t c = 0; c < ng; ++c) {
+            const float *B = blocks[t] + c * b * b;
+            for (int k = 0; k < b; ++k)
+                for (int j = 0; j < b; ++j) {
+                    const float v = B[k * b + j];
+                    const float hi = tf32_rna(v), lo = tf32_rna(v - hi);
+                    uf[c * ublk + harp::umma_block_index(k, j, up)] = hi;
+                    uf[c * ublk + harp::umma_block_index(up + k, j, up)] = lo;
+                    ui[c * ublk + harp::umma_block_index(j, k, up)] = hi;
+                    ui[c * ublk + harp::umma_block_index(up + j, k, up)] = lo;
                 }
         }
     }
@@ -369,6 +415,10 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
         p->dev.st[t].pfwd = base + poff[t];
         p->dev.st[t].pinv = base + poff[t] + static_cast<size_t>(d / b) * pass_jpad(b) * pass_kp(b);
         p->dev.st[t].had = all_sylvester(b, d / b, blocks[t]) ? 1 : 0;
+        const int up = umma_up(b);
+        p->dev.st[t].up = up;
+        p->dev.st[t].ufwd = base + uoff[t];
+        p->dev.st[t].uinv = base + uoff[t] + static_cast<size_t>(d / b) * 2 * up * up;
     }
     *out = p;
     return HARP_OK;
@@ -396,9 +446,7 @@ int harp_theta_blocks(int b, int64_t n_groups, const int8_t *theta, float theta_
 int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float theta_scale,
                          const float *base, void *stream) {
     if (!plan || stage < 0 || stage >= plan->m) return HARP_ERR_INVALID_ARG;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HARP_ERR_CUDA; }
-    if (dev != plan->device) return HARP_ERR_INVALID_ARG;   // the plan's memory lives on its own device
+    if (int dv = plans_on_current_device(plan)) return dv;   // the plan's memory lives on its own device
     harp::StageDev &sd = plan->dev.st[stage];
     const int b = sd.b;
     const int64_t ng = plan->d / b;
@@ -412,6 +460,9 @@ int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float
     o.pinv = const_cast<float *>(sd.pinv);
     o.jp = sd.jpad;
     o.kp = sd.kp;
+    o.ufwd = const_cast<float *>(sd.ufwd);
+    o.uinv = const_cast<float *>(sd.uinv);
+    o.up = sd.up;
     st = cuda_status(harp::launch_theta_blocks(b, ng, theta, theta_scale, base, o, stream));
     if (st == HARP_OK) sd.had = 0;
     return st;
@@ -480,12 +531,14 @@ int harp_workspace_size(harp_plan_t left, harp_plan_t right, int64_t rows, int64
 }
 
 static bool valid_dtype(int t) { return t == HARP_F32 || t == HARP_BF16; }
+
 static size_t dtype_size(int t) { return t == HARP_F32 ? 4 : 2; }
 
 int harp_rotate(harp_plan_t plan, int side, int dir, const void *in, int in_dtype, void *out,
                 int out_dtype, int64_t rows, int64_t cols, int64_t ld_in, int64_t ld_out,
                 void *stream) {
     if (!plan) return HARP_ERR_INVALID_ARG;
+    if (int dv = plans_on_current_device(plan)) return dv;
     if (side != HARP_RIGHT && side != HARP_LEFT) return HARP_ERR_INVALID_ARG;
     if (dir != HARP_FWD && dir != HARP_INV) return HARP_ERR_INVALID_ARG;
     if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return HARP_ERR_INVALID_ARG;
@@ -554,7 +607,9 @@ static bool use_passes(harp_plan_t left, harp_plan_t right, harp_codebook_t cb) 
 static int check_pair(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int64_t rows,
                       int64_t cols, void *workspace, size_t ws_bytes) {
     if (!right || !cb) return HARP_ERR_INVALID_ARG;
-    int st = check_codec(cb, rows, cols);
+    int st = plans_on_current_device(left, right);
+    if (st) return st;
+    st = check_codec(cb, rows, cols);
     if (st) return st;
     if (right->d != cols) return HARP_ERR_SHAPE;
     if (left && left->d != rows) return HARP_ERR_SHAPE;
@@ -634,6 +689,7 @@ int harp_requantize(harp_plan_t right, harp_codebook_t cb_in, const uint8_t *cod
                     void *restored_out, harp_codebook_t cb_out, uint8_t *codes_out,
                     uint16_t *scales_out, void *stream) {
     if (!right || !cb_in || !cb_out) return HARP_ERR_INVALID_ARG;
+    if (int dv = plans_on_current_device(right)) return dv;
     if (mid_dtype != HARP_F32 && mid_dtype != HARP_BF16 && mid_dtype != HARP_F16) return HARP_ERR_INVALID_ARG;
     int st = check_codec(cb_in, rows, cols);
     if (st == HARP_OK) st = check_codec(cb_out, rows, cols);
@@ -689,6 +745,17 @@ int harp_pass_fma(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int p
     if (f < 0) return HARP_ERR_INVALID_ARG;
     *fma = f;
     return HARP_OK;
+}
+
+int harp_set_block_stages(int mode) {
+    if (mode < HARP_BLOCK_STAGES_AUTO || mode > HARP_BLOCK_STAGES_FFMA) return HARP_ERR_INVALID_ARG;
+    harp::set_block_stages(mode);
+    return HARP_OK;
+}
+
+int harp_fault_status(unsigned int *flags) {
+    if (!flags) return HARP_ERR_INVALID_ARG;
+    return cuda_status(harp::pass_fault_status(flags));
 }
 
 int harp_set_pass_events(void *const *events, int n) {

@@ -6,6 +6,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "harp.h"
 
 namespace harp {
@@ -34,7 +36,25 @@ struct StageDev {
     // Hadamard matrix (fp32 entries +-1/sqrt(b), b a power of two): the pass
     // kernels then apply the stage as a fast Walsh-Hadamard butterfly.
     int had;
+    // The same blocks as tensor-core operands for the pass kernels' 3xTF32
+    // stages (split-precision products on tcgen05.mma kind::tf32): up = b
+    // rounded up to 16; per group 2*up x up floats, K-major "core matrix"
+    // order (8 operand rows x 4 inputs per 128-byte unit):
+    //   float index (kk/4)*8*up + (n/8)*32 + (n%8)*4 + kk%4
+    // for operand row n (output) and input kk. Rows n < up hold the
+    // tf32-rounded coefficients (hi), rows up + n the tf32-rounded remainders
+    // (lo = coefficient - hi). ufwd: output k, input j -> B[k][j]; uinv:
+    // output j, input k -> B[k][j] (the transposed blocks). Zero in padding.
+    int up;
+    const float *ufwd;
+    const float *uinv;
 };
+
+// Operand float index of (row n, input kk) in a tensor-core block of
+// padded size up (see StageDev).
+__host__ __device__ inline int umma_block_index(int n, int kk, int up) {
+    return (kk >> 2) * 8 * up + (n >> 3) * 32 + (n & 7) * 4 + (kk & 3);
+}
 
 struct PlanDev {
     int64_t d;
@@ -120,6 +140,14 @@ int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q
                     const uint8_t *codes, const uint16_t *scales, void *out, int out_dtype,
                     float *ws, void *stream);
 
+// Implementation of the pass kernels' block stages (harp_set_block_stages).
+enum BlockStages { BLOCK_STAGES_AUTO = 0, BLOCK_STAGES_TC = 1, BLOCK_STAGES_FFMA = 2 };
+void set_block_stages(int mode);
+
+// Reads and clears the pass kernels' record of bounded waits that ran out
+// on the current device (cudaError_t; synchronous).
+int pass_fault_status(unsigned *flags);
+
 // Timing hook of the pass launchers (harp_set_pass_events): when n > 0,
 // every fused call records events[0] before its first pass and events[k+1]
 // after pass k (k + 1 < n). Per calling thread.
@@ -137,6 +165,9 @@ struct ThetaOut {
     float *pinv;    // [(c jp + k) kp + j] = B[k][j]
     int jp;
     int kp;
+    float *ufwd;    // tensor-core operand blocks (StageDev::ufwd / uinv), up = padded size
+    float *uinv;
+    int up;
 };
 size_t theta_smem_bytes(int b);
 int launch_theta_blocks(int b, int64_t n_groups, const int8_t *theta, double scale,
@@ -164,6 +195,13 @@ struct ShortLaunch {
 };
 bool short_ok(const PlanDev &P, int mode, int in_bits);
 int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &L, void *stream);
+
+// A plan's blocks live in device memory of the device that was current when
+// it was created; a launch from another device would read them through a
+// foreign address. HARP_OK when every non-null plan belongs to the current
+// device, HARP_ERR_INVALID_ARG otherwise (HARP_ERR_CUDA without a device).
+// Every entry point that launches checks this before anything else.
+int plans_on_current_device(harp_plan_t a, harp_plan_t b = nullptr);
 
 // Vectors per CTA the whole-vector kernel uses for this plan and epilogue
 // (0 if a vector does not fit in shared memory).

@@ -37,6 +37,7 @@
 
 #include "harp_internal.h"
 #include "harp_quant_dev.cuh"
+#include "harp_tc.cuh"
 
 namespace harp {
 namespace {
@@ -49,6 +50,8 @@ constexpr int MAXPS = 12;             // stages (both sides) in one pass
 constexpr int TILE_MAX = 16384;       // tile elements
 constexpr int SMEM_BUDGET = 232448;    // bytes per CTA (opt-in maximum): two tile buffers
 constexpr int GPAD = 4;               // floats between coefficient slots
+constexpr int TC_MIN_SMEM = 120 * 1024;
+constexpr int MAX_SLOTS_HOST = 8;     // tensor-core slots at the narrowest blocks (512 / 64)  // shared memory of a tensor-core CTA: more than half an SM's
 
 // Division by a fixed divisor d >= 1 as a multiply-high and a shift (exact
 // for dividends below 2^31): sh = ceil(log2 d), mul = 2^32 (2^sh - d) / d + 1.
@@ -100,6 +103,16 @@ struct PStage {
     int64_t s;        // global stride of the digit
     const float *coef;  // [d/b][jpad][kp]
     int had;          // every block is the normalised Sylvester Hadamard: butterfly, no coefficients
+    // tensor-core stages (the tcgen05 build): the stage as a batch of
+    // split-precision products, one MMA "instance" per (group, block of mb
+    // vectors): D[v][k] = sum_j x_v[j] B[k][j], K = N = up.
+    int up;           // b rounded up to 16
+    int mb;           // vectors per instance: 128, or 64 (two instances share TMEM columns)
+    int nvb;          // vector blocks of mb
+    int nslots;       // TMEM slots of 4*up columns (A hi, A lo, D)
+    int ucoff;        // byte offset of the stage's operand blocks in the coefficient area
+    const float *ucoef; // [d/b][2 up up] operand blocks (forward or inverse)
+    FDiv f_nvb, f_sig;  // divisions by nvb and sig
 };
 
 struct PassDesc {
@@ -121,6 +134,11 @@ struct PassDesc {
     int coef_base;      // float offset of the coefficient area
     int coef_floats;
     int tab_base;       // float offset of the index tables (rows, then cols)
+    int coef_single;    // tensor-core build: one coefficient area at coef_base, refilled stage by stage
+    int in_bulk;        // tensor-core build: 0 = cp.async, 1 = one contiguous tile (bulk copy),
+                        // 2 = one bulk copy per tile row of in_row_bytes
+    int in_row_bytes;
+    int tc_base;        // tensor-core build: float offset of the TMEM address slot and the mbarrier
     int smem_bytes;
     int sign_at_store;  // inverse: signs after the stages
     int bins;           // quantising pass: Lloyd-Max codes by the 64-bin table (exact for these midpoints)
@@ -406,6 +424,203 @@ __device__ __noinline__ void stage_rounds(float *T, const float *C, const PStage
     stage_run<8, true>(T, C, S, A, Bv, NV, warp, lane);
 }
 
+// ------------------------------------------------------------ tensor-core stage
+
+// Device record of bounded waits that ran out (bit 0: an MMA batch never
+// completed). Kernels never trap; the host reads this with
+// harp_fault_status.
+__device__ unsigned int g_pass_fault;
+
+constexpr int TMEM_COLS = 512;
+constexpr long long MMA_WAIT_LIMIT = 1ll << 30;   // SM cycles (about half a second)
+
+// One block stage on the tensor cores (tcgen05.mma kind::tf32, 3xTF32):
+// every instance (group g, block of mb vectors) is the product
+//     D[v][n] = sum_j x_v[j] * Bop[n][j],   n < 2*UP,  j < UP,
+// of the vectors' inputs (rows of A, in TMEM: tf32 hi in UP columns, the
+// tf32 remainder lo in the next UP) and the group's operand block (2*UP rows:
+// the tf32 coefficients, then their remainders; shared memory). Per 8-input
+// step one MMA multiplies A_hi by all 2*UP rows (N = 2*UP) and one adds A_lo
+// times the hi rows (N = UP) into the first half, so the output is
+//     y_v[k] = D[v][k] + D[v][UP + k]
+//            = sum_j (x_hi b_hi + x_lo b_hi) + sum_j x_hi b_lo,
+// x*b to about 2^-22 relative with fp32 accumulation.
+//
+// TMEM (512 columns) holds SLOTS slots of 4*UP columns (A hi | A lo | D); a
+// slot carries one instance (mb = 128) or two (mb = 64, lanes 0-15 and 16-31
+// of every 32-lane quarter). A stage runs in rounds of up to SLOTS slots:
+//   1. every warp splits and stores its items (slot, 16-column chunk) of its
+//      TMEM quarter (warp w serves lanes 32*(w%4)..+31), all before one
+//      tcgen05.wait::st, then arrives on each touched slot's "A full"
+//      mbarrier (the 4*UP/16 items of a slot arrive with AFULL_COUNT in
+//      total);
+//   2. warps 0..3 (one elected thread each) take every fourth slot: wait for
+//      its A, issue its MMAs, commit to its "D full" mbarrier;
+//   3. every warp waits for the slots of its items, loads their D with one
+//      tcgen05.wait::ld, and writes y back into the tile in place.
+// The MMAs of early slots run while later slots are still being stored and
+// earlier ones read back. Inputs past b are zeros, outputs past b are
+// dropped. Returns false when a wait ran out (the stage is then abandoned).
+constexpr int MAX_SLOTS = TMEM_COLS / 64;   // slots at UP = 16
+constexpr int AFULL_COUNT = 48;             // items per slot (4, 8, 12, 16) all divide it
+
+// The stage mbarriers and the parity each slot's next phase will have
+// (bit s; every barrier completes exactly once per round that uses it).
+struct TcBars {
+    uint64_t *afull;    // [MAX_SLOTS] A of the slot stored (count AFULL_COUNT)
+    uint64_t *dfull;    // [MAX_SLOTS] MMAs of the slot done (one commit)
+    uint32_t par;       // phase parity of slot s in bit s (the same for both barriers)
+};
+
+template <int UP, bool EXACT>
+__device__ __forceinline__ bool stage_tc(float *T, const float *Cs, const PStage &S, int A, int Bv, int NV,
+                                         int warp, int lane, uint32_t tmem, TcBars &bars, uint64_t *cbar,
+                                         uint32_t cpar) {
+    bool coef_ready = false;
+    constexpr int NCH = UP / 16;                  // 16-column chunks per slot
+    constexpr int SLOTS = TMEM_COLS / (4 * UP);
+    constexpr int IPW = (SLOTS * NCH + 3) / 4;    // items per warp in a round (at most)
+    const int q = warp & 3, wu = warp >> 2;
+    const int MB = S.mb, per = (MB == 64) ? 2 : 1;
+    const int ninst = S.G * S.nvb;
+    const int ipr = SLOTS * per;                  // instances per round
+    const int step = S.sig * A;
+    const uint32_t lane_q = static_cast<uint32_t>(32 * q) << 16;
+    const int h = (MB == 64) ? (lane >> 4) : 0;
+    const int vlane = (MB == 128) ? 32 * q + lane : 16 * q + (lane & 15);
+
+    // tile address of this lane's vector of instance `inst` (element j at + j*step)
+    auto lane_base = [&](int inst, bool &ok) -> int {
+        const int g = static_cast<int>(fdiv(static_cast<unsigned>(inst), S.f_nvb));
+        const int vb = inst - g * S.nvb;
+        const int v = vb * MB + vlane;
+        ok = inst < ninst && v < NV;
+        const int gg = ok ? g : 0, vv = ok ? v : 0;
+        const int hi = static_cast<int>(fdiv(static_cast<unsigned>(gg), S.f_sig));
+        const int base = hi * (S.b * S.sig) + (gg - hi * S.sig);
+        return base * A + vv * Bv;
+    };
+
+    for (int i0 = 0; i0 < ninst; i0 += ipr) {
+        const int nsl = min(SLOTS, (ninst - i0 + per - 1) / per);
+        const int nit = nsl * NCH;                // items per quarter this round
+        tc::fence_after_sync();                   // the previous round's TMEM reads are done
+        // ---- 1+2. A: split and store this warp's items; the warp of
+        // quarter 0 that writes a slot's first chunk then waits for the
+        // slot's other items and issues its MMAs right away, so the tensor
+        // cores start on early slots while later ones are still written
+        bool good = true;
+        constexpr uint32_t id1 = tc::idesc_tf32(128, 2 * UP), id2 = tc::idesc_tf32(128, UP);
+        constexpr uint32_t id1h = tc::idesc_tf32(64, 2 * UP), id2h = tc::idesc_tf32(64, UP);
+#pragma unroll
+        for (int u = 0; u < IPW; ++u) {
+            const int it = wu + 4 * u;
+            if (it >= nit) continue;
+            const int sl = it / NCH, c = it - sl * NCH;
+            {
+                bool ok;
+                const int p = lane_base(i0 + sl * per + h, ok);
+                const float *xp = T + p + 16 * c * step;
+                // every load is unconditional (inputs past b re-read input
+                // b-1, lanes without a vector read the tile's first group) and
+                // selected afterwards, so the 16 loads issue back to back
+                float xv[16], hv[16], lv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int j = EXACT ? i : min(16 * c + i, S.b - 1) - 16 * c;
+                    xv[i] = xp[j * step];
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const bool in = EXACT ? ok : (ok && 16 * c + i < S.b);
+                    tc::split_tf32(in ? xv[i] : 0.0f, hv[i], lv[i]);
+                }
+                const uint32_t ta = tmem + lane_q + static_cast<uint32_t>(sl * 4 * UP + 16 * c);
+                tc::st16(ta, hv);
+                tc::st16(ta + UP, lv);
+            }
+            tc::wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars.afull[sl], AFULL_COUNT / (4 * NCH));
+            if (q == 0 && c == 0) {
+                if (!coef_ready) {
+                    // this tile's operand blocks of the stage
+                    coef_ready = tc::mbar_wait_bounded(cbar, cpar, MMA_WAIT_LIMIT);
+                    good = good && coef_ready;
+                }
+                const bool ready = tc::mbar_wait_bounded(&bars.afull[sl], (bars.par >> sl) & 1u, MMA_WAIT_LIMIT);
+                good = good && ready;
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    if (ready && coef_ready) {
+                        const uint32_t cbase = tc::smem_u32(Cs) + static_cast<uint32_t>(S.ucoff);
+                        for (int hh = 0; hh < per; ++hh) {
+                            const int inst = i0 + sl * per + hh;
+                            if (inst >= ninst) continue;
+                            const int g = static_cast<int>(fdiv(static_cast<unsigned>(inst), S.f_nvb));
+                            const uint32_t a = tmem + (static_cast<uint32_t>(16 * hh) << 16) +
+                                               static_cast<uint32_t>(sl * 4 * UP);
+                            const uint32_t d = a + 2 * UP;
+                            const uint32_t bsm = cbase + static_cast<uint32_t>(g * 8 * UP * UP);
+#pragma unroll
+                            for (int st = 0; st < UP / 8; ++st) {
+                                const uint64_t bd =
+                                    tc::smem_desc(bsm + static_cast<uint32_t>(st * 64 * UP), 32 * UP, 128);
+                                tc::mma_tf32_ts(d, a + 8 * st, bd, MB == 128 ? id1 : id1h, st > 0);
+                                tc::mma_tf32_ts(d, a + UP + 8 * st, bd, MB == 128 ? id2 : id2h, 1u);
+                            }
+                        }
+                    }
+                    tc::mma_commit(&bars.dfull[sl]);
+                }
+                __syncwarp();
+            }
+        }
+        // ---- 3. D: for each item of this warp, wait for its slot, load both
+        // halves of D, y back into the tile
+#pragma unroll
+        for (int u = 0; u < IPW; ++u) {
+            const int it = wu + 4 * u;
+            if (it >= nit) continue;
+            const int sl = it / NCH, c = it - sl * NCH;
+            good = tc::mbar_wait_bounded(&bars.dfull[sl], (bars.par >> sl) & 1u, MMA_WAIT_LIMIT) && good;
+            tc::fence_after_sync();
+            const uint32_t td = tmem + lane_q + static_cast<uint32_t>(sl * 4 * UP + 2 * UP + 16 * c);
+            float da[16], db[16];
+            tc::ld16(td, da);
+            tc::ld16(td + UP, db);
+            tc::wait_ld();
+            if (!good) continue;
+            bool ok;
+            const int p = lane_base(i0 + sl * per + h, ok);
+            float *yp = T + p + 16 * c * step;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const bool out = EXACT ? ok : (ok && 16 * c + i < S.b);
+                if (out) yp[i * step] = da[i] + db[i];
+            }
+        }
+        bars.par ^= (1u << nsl) - 1u;             // slots 0..nsl-1 completed one phase each
+        tc::fence_before_sync();
+        if (__syncthreads_or(good ? 0 : 1)) return false;   // slots free, tile complete
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool stage_tc_any(float *T, const float *Cs, const PStage &S, int A, int Bv, int NV,
+                                             int warp, int lane, uint32_t tmem, TcBars &bars, uint64_t *cbar,
+                                             uint32_t cpar) {
+    const bool ex = (S.b == S.up);
+    switch (S.up) {
+        case 16: return ex ? stage_tc<16, true>(T, Cs, S, A, Bv, NV, warp, lane, tmem, bars, cbar, cpar)
+                           : stage_tc<16, false>(T, Cs, S, A, Bv, NV, warp, lane, tmem, bars, cbar, cpar);
+        case 32: return stage_tc<32, false>(T, Cs, S, A, Bv, NV, warp, lane, tmem, bars, cbar, cpar);
+        case 48: return stage_tc<48, false>(T, Cs, S, A, Bv, NV, warp, lane, tmem, bars, cbar, cpar);
+        default: return stage_tc<64, false>(T, Cs, S, A, Bv, NV, warp, lane, tmem, bars, cbar, cpar);
+    }
+}
+
 // ------------------------------------------------------------ prologue / epilogue
 
 
@@ -619,7 +834,7 @@ __device__ __forceinline__ Buf buf_of(float *sm, const PassDesc &D, int b) {
     Buf B;
     float *base = sm + D.tile_floats + b * D.buf_floats;
     B.T = sm;
-    B.C = base;
+    B.C = D.coef_single ? sm + D.coef_base : base;
     B.rin = reinterpret_cast<int64_t *>(base + D.tab_base);
     B.rout = B.rin + Er;
     B.rtab = reinterpret_cast<int *>(B.rout + Er);
@@ -692,6 +907,67 @@ __device__ __forceinline__ void issue_coefs(const PassDesc &D, const Tabs &tb, f
             for (int o = lane; o < cpg; o += 32) cp_async16(dst + 4 * o, src + 4 * o);
         }
     }
+}
+
+// Tensor-core operand blocks of stage u of a tile into the (single)
+// coefficient area, by one warp: each of the tile's groups gets its global
+// group's 2*up x up block (contiguous in global and shared memory) by one
+// bulk copy; `bar` completes when all have landed.
+__device__ __forceinline__ void issue_coefs_bulk(const PassDesc &D, const Tabs &tb, float *C, int u, uint64_t *bar,
+                                                 int lane) {
+    const PStage &S = D.st[u];
+    if (S.had) return;
+    const int fpg = 2 * S.up * S.up;
+    if (lane == 0) tc::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(S.G * fpg * 4));
+    __syncwarp();
+    const int *tab = S.axis == 0 ? tb.rtab : tb.ctab;
+    float *area = C + S.ucoff / 4;
+    for (int gi = lane; gi < S.G; gi += 32) {
+        const int c = global_group(S, tab, gi);
+        tc::bulk_g2s(area + gi * fpg, S.ucoef + static_cast<int64_t>(c) * fpg, static_cast<uint32_t>(fpg * 4), bar);
+    }
+}
+
+// The next tile's input by bulk copies (one warp), completing on `bar`: the
+// whole tile when the input is a workspace in this pass's tile-major order,
+// else one copy per tile row (rows of contiguous bf16 values or packed codes).
+template <int PRO>
+__device__ __forceinline__ void issue_input_bulk(const PassDesc &D, const QuantDev &Q, const Tabs &tb, void *S,
+                                                 unsigned t, uint64_t *bar, int lane) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E;
+    if (D.in_bulk == 1) {
+        const uint32_t bytes = static_cast<uint32_t>(Er * Ec * 4);
+        if (lane == 0) {
+            tc::mbar_arrive_expect_tx(bar, bytes);
+            tc::bulk_g2s(S, static_cast<const float *>(D.in) + static_cast<int64_t>(t) * Er * Ec, bytes, bar);
+        }
+        return;
+    }
+    const int rb = D.in_row_bytes;
+    if (lane == 0) tc::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(Er * rb));
+    __syncwarp();
+    for (int tr = lane; tr < Er; tr += 32) {
+        const char *src;
+        if constexpr (PRO == PRO_CODES)
+            src = reinterpret_cast<const char *>(D.in_codes) + static_cast<int64_t>(tb.rtab[tr]) * (D.cols * Q.bits / 8) +
+                  static_cast<int64_t>(tb.ctab[0]) * Q.bits / 8;
+        else
+            src = static_cast<const char *>(D.in) + (tb.rin[tr] + tb.cin[0]) * 2;
+        tc::bulk_g2s(static_cast<char *>(S) + tr * rb, src, static_cast<uint32_t>(rb), bar);
+    }
+}
+
+// Scales of the next codes tile (one register per thread), as issue_input
+// loads them.
+__device__ __forceinline__ float load_tile_scales(const PassDesc &D, const QuantDev &Q, const Tabs &tb, int tid) {
+    const int Er = D.ax[0].E, Ec = D.ax[1].E, ngt = Ec / Q.group;
+    float sc = 0.0f;
+    if (tid < Er * ngt) {
+        const int tr = static_cast<int>(fdiv(static_cast<unsigned>(tid), D.f_ngt)), q = tid - tr * ngt;
+        sc = __half2float(__ushort_as_half(__ldg(D.in_scales + static_cast<int64_t>(tb.rtab[tr]) * (D.cols / Q.group) +
+                                                 tb.ctab[0] / Q.group + q)));
+    }
+    return sc;
 }
 
 constexpr int MAXCH = 8;   // 32-code chunks per row of a quantised tile (Ec <= 256)
@@ -815,7 +1091,8 @@ __device__ __forceinline__ void convert_input(const PassDesc &D, const QuantDev 
 enum StageSet {
     SS_ALL = 0,    // Walsh-Hadamard butterflies and all block widths
     SS_BLOCKS = 1, // block stages of any width, no butterfly
-    SS_K16 = 2     // only block stages of exactly 16 outputs and inputs
+    SS_K16 = 2,    // only block stages of exactly 16 outputs and inputs
+    SS_TC = 3      // block stages on the tensor cores (3xTF32), Walsh-Hadamard butterflies
 };
 
 template <int PRO, int EPI, int SS>
@@ -833,6 +1110,31 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
     const unsigned ntiles = static_cast<unsigned>(D.ax[0].nt * D.ax[1].nt);
     unsigned t = blockIdx.x;
     if (t >= ntiles) return;
+    constexpr bool TC = (SS == SS_TC);
+    uint32_t tmem = 0;
+    TcBars bars{nullptr, nullptr, 0u};
+    uint64_t *cbar = nullptr, *ibar = nullptr;
+    if constexpr (TC) {
+        // the whole TMEM of the SM (one CTA per SM), the per-slot mbarriers
+        // of the tensor-core stages, one mbarrier per stage for its operand
+        // blocks and one for the next tile's input (bulk copies)
+        uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + D.tc_base);
+        bars.afull = reinterpret_cast<uint64_t *>(sm + D.tc_base + 2);
+        bars.dfull = bars.afull + MAX_SLOTS;
+        cbar = bars.dfull + MAX_SLOTS;
+        ibar = cbar + MAXPS;
+        if (warp == 0) tc::tmem_alloc(tslot, TMEM_COLS);
+        if (tid < MAX_SLOTS) {
+            tc::mbar_init(&bars.afull[tid], AFULL_COUNT);
+            tc::mbar_init(&bars.dfull[tid], 1);
+        }
+        if (tid < MAXPS) tc::mbar_init(&cbar[tid], 1);
+        if (tid == 0) tc::mbar_init(ibar, 1);
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        tmem = *tslot;
+    }
     if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
         // a quantising pass decodes nothing: the level slots hold the bin table
         const int K = 1 << Q.bits;
@@ -854,16 +1156,32 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
         const Buf B0 = buf_of(sm, D, 0);
         build_tables(D, B0, rloc, cloc, t, ld, tid);
         __syncthreads();
-        sc_next = issue_input<PRO>(D, Q, B0.tb, S, tid);
-        issue_coefs(D, B0.tb, B0.C, warp, lane);
+        if constexpr (TC) {
+            if (D.in_bulk) {
+                if (warp == 0) issue_input_bulk<PRO>(D, Q, B0.tb, S, t, ibar, lane);
+                sc_next = (PRO == PRO_CODES) ? load_tile_scales(D, Q, B0.tb, tid) : 0.0f;
+            } else {
+                sc_next = issue_input<PRO>(D, Q, B0.tb, S, tid);
+            }
+            if (warp == 1)
+                for (int u = 0; u < D.nst; ++u) issue_coefs_bulk(D, B0.tb, B0.C, u, &cbar[u], lane);
+        } else {
+            sc_next = issue_input<PRO>(D, Q, B0.tb, S, tid);
+            issue_coefs(D, B0.tb, B0.C, warp, lane);
+        }
         cp_async_commit();
         cp_async_wait_all();
+        if constexpr (TC) {
+            if (D.in_bulk && !tc::mbar_wait_bounded(ibar, 0u, MMA_WAIT_LIMIT) && tid == 0) atomicOr(&g_pass_fault, 2u);
+        }
         if (PRO == PRO_CODES && tid < Er * (Ec / Q.group)) B0.ssc[tid] = sc_next;
         __syncthreads();
         convert_input<PRO>(D, Q, B0.tb, S, T, B0.ssc, lev, load_signs, tid, warp, lane);
         __syncthreads();
     }
 
+    bool fault = false, fault_more = false;
+    int fault_k = 0, fault_u = 0;
     for (int k = 0; t < ntiles; ++k, t += gridDim.x) {
         const Buf B = buf_of(sm, D, k & 1);
         const unsigned tn = t + gridDim.x;
@@ -872,8 +1190,13 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
         if (more) {
             build_tables(D, Bn, rloc, cloc, tn, ld, tid);
             __syncthreads();
-            sc_next = issue_input<PRO>(D, Q, Bn.tb, S, tid);
-            issue_coefs(D, Bn.tb, Bn.C, warp, lane);
+            if (TC && D.in_bulk) {
+                if (warp == 0) issue_input_bulk<PRO>(D, Q, Bn.tb, S, tn, ibar, lane);
+                sc_next = (PRO == PRO_CODES) ? load_tile_scales(D, Q, Bn.tb, tid) : 0.0f;
+            } else {
+                sc_next = issue_input<PRO>(D, Q, Bn.tb, S, tid);
+            }
+            if constexpr (!TC) issue_coefs(D, Bn.tb, Bn.C, warp, lane);
             cp_async_commit();
         }
 
@@ -881,7 +1204,32 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
             const PStage &S = D.st[u];
             const bool rows = (S.axis == 0);
             const int A = rows ? TCp : 1, Bv = rows ? 1 : TCp, NV = rows ? Ec : Er;
-            if constexpr (SS == SS_K16) {
+            if constexpr (SS == SS_TC) {
+                if (S.had) {
+                    switch (S.b) {
+                        case 2: stage_fwht<2>(T, S, A, Bv, NV, warp, lane); break;
+                        case 4: stage_fwht<4>(T, S, A, Bv, NV, warp, lane); break;
+                        case 8: stage_fwht<8>(T, S, A, Bv, NV, warp, lane); break;
+                        case 16: stage_fwht<16>(T, S, A, Bv, NV, warp, lane); break;
+                        default: stage_fwht<32>(T, S, A, Bv, NV, warp, lane); break;
+                    }
+                } else {
+                    // the stage's issuing warps wait for this tile's operand
+                    // blocks (bulk copies issued after the previous tile's stage u)
+                    if (!stage_tc_any(T, B.C, S, A, Bv, NV, warp, lane, tmem, bars, &cbar[u],
+                                      static_cast<uint32_t>(k & 1))) {
+                        fault = true;
+                        fault_more = more;
+                        fault_k = k;
+                        fault_u = u;
+                        break;
+                    }
+                    // the blocks are consumed: bring the next tile's (the stage
+                    // ended on a CTA barrier, so the next stage needs no other)
+                    if (more && warp == 1) issue_coefs_bulk(D, Bn.tb, Bn.C, u, &cbar[u], lane);
+                    continue;
+                }
+            } else if constexpr (SS == SS_K16) {
                 stage_run<16, false, true>(T, B.C, S, A, Bv, NV, warp, lane);
             } else {
                 if (SS == SS_ALL && S.had) {
@@ -900,6 +1248,7 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
             }
             __syncthreads();
         }
+        if (fault) break;
 
         if constexpr (EPI == EPI_QUANT || EPI == EPI_QUANT_F32) {
             constexpr bool F = (EPI == EPI_QUANT_F32);
@@ -914,10 +1263,46 @@ pass_kernel(const __grid_constant__ PassDesc D, const __grid_constant__ QuantDev
 
         if (more) {
             cp_async_wait_all();
+            if constexpr (TC) {
+                if (D.in_bulk && !tc::mbar_wait_bounded(ibar, static_cast<uint32_t>((k + 1) & 1), MMA_WAIT_LIMIT) &&
+                    tid == 0)
+                    atomicOr(&g_pass_fault, 2u);
+            }
             if (PRO == PRO_CODES && tid < Er * (Ec / Q.group)) Bn.ssc[tid] = sc_next;
             __syncthreads();
             convert_input<PRO>(D, Q, Bn.tb, S, T, Bn.ssc, lev, load_signs, tid, warp, lane);
+            // the staging buffer's reads are ordered before the next bulk copy into it
+            if constexpr (TC) tc::fence_proxy_async();
             __syncthreads();
+        }
+    }
+
+    if constexpr (TC) {
+        // copies still in flight land before the CTA leaves; an abandoned
+        // batch gets one more bounded wait before its TMEM is released
+        cp_async_wait_all();
+        if (fault) {
+            // every slot's MMAs of the abandoned round (each slot was committed)
+            if (tid == 0) atomicOr(&g_pass_fault, 1u);
+            if (tid < MAX_SLOTS) tc::mbar_wait_bounded(&bars.dfull[tid], (bars.par >> tid) & 1u, MMA_WAIT_LIMIT);
+        }
+        // bulk copies for the next tile issued before the fault land before the
+        // CTA's shared memory is released
+        if (fault) {
+            const uint32_t cp = static_cast<uint32_t>(fault_k & 1), np = cp ^ 1u;
+            // this tile's blocks of the stages not reached yet, and the next
+            // tile's input and blocks issued before the fault
+            if (tid >= fault_u && tid < D.nst && !D.st[tid].had) tc::mbar_wait_bounded(&cbar[tid], cp, MMA_WAIT_LIMIT);
+            if (fault_more) {
+                if (tid == 0 && D.in_bulk) tc::mbar_wait_bounded(ibar, np, MMA_WAIT_LIMIT);
+                if (tid < fault_u && !D.st[tid].had) tc::mbar_wait_bounded(&cbar[tid], np, MMA_WAIT_LIMIT);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        if (warp == 0) {
+            tc::fence_after_sync();
+            tc::tmem_dealloc(tmem, TMEM_COLS);
         }
     }
 }
@@ -1004,20 +1389,73 @@ int tcp_of(int Ec) { return (Ec % 2 == 0) ? Ec + 1 : Ec; }
 // dequantised levels.
 struct SmemLayout {
     int tile_floats, coef_floats, tab_base, buf_floats, stage_base, loc_base, lev_base, total_floats;
+    int coef_single, coef_base, tc_base;
 };
+
+// Which implementation the block stages of the pass kernels use (process-
+// wide, harp_set_block_stages): automatic, always the tensor-core build, or
+// always the FFMA builds.
+int g_block_stage_mode = BLOCK_STAGES_AUTO;
+
+// Whether a pass applying L[iL:jL] and R[iR:jR] runs the tensor-core build.
+// It must have a block stage that is not a Walsh-Hadamard butterfly; then,
+// automatically, only when one of its blocks is wider than 32: measured on
+// the B200 (4096x4096, 4096x11008, 8192x28672 workloads), the tcgen05 stages
+// beat the FFMA stages on the 43-wide blocks (a pass with them 17 % faster)
+// and lose on blocks of 7, 16 and 32 (passes 10-25 % slower), where the
+// per-stage round trip through TMEM costs more than the FFMAs it replaces.
+bool pass_uses_tc(const PlanInput &in, int iL, int jL, int iR, int jR) {
+    if (g_block_stage_mode == BLOCK_STAGES_FFMA) return false;
+    bool blocks = false, wide = false;
+    for (int t = iL; in.L && t < jL; ++t)
+        if (!stage_is_fwht(in.L->st[t])) {
+            blocks = true;
+            wide = wide || in.L->st[t].b > 32;
+        }
+    for (int t = iR; t < jR; ++t)
+        if (!stage_is_fwht(in.R->st[t])) {
+            blocks = true;
+            wide = wide || in.R->st[t].b > 32;
+        }
+    return blocks && (wide || g_block_stage_mode == BLOCK_STAGES_TC);
+}
+
+// Tensor-core operand bytes of the stages [i, j) of one side for a tile
+// with E coordinates along that side: (E / b) groups of 2*up*up floats.
+int stage_ucoef_floats(const PlanDev *pl, int i, int j, int E) {
+    int f = 0;
+    for (int t = i; t < j; ++t) {
+        const StageDev &s = pl->st[t];
+        if (!stage_is_fwht(s)) f += (E / s.b) * 2 * s.up * s.up;
+    }
+    return f;
+}
 
 SmemLayout smem_layout(const PlanInput &in, int iL, int jL, int iR, int jR, int Er, int Ec) {
     SmemLayout L;
-    L.tile_floats = (Er * tcp_of(Ec) + 3) & ~3;
-    L.coef_floats = (in.L ? stage_coef_floats(in.L, iL, jL, Er) : 0) + stage_coef_floats(in.R, iR, jR, Ec);
-    L.tab_base = (L.coef_floats + 1) & ~1;
-    int b = L.tab_base + 2 * Er + 2 * Er + Er + 3 * Ec + Er + Ec;   // rin, rout (int64), rtab, ctab, cin, cout, signs
-    if (Ec % in.group == 0) b += Er * (Ec / in.group);            // scales of a codes tile
-    L.buf_floats = (b + 3) & ~3;
-    L.stage_base = L.tile_floats + 2 * L.buf_floats;
+    L.coef_single = pass_uses_tc(in, iL, jL, iR, jR) ? 1 : 0;
+    L.tile_floats = (Er * tcp_of(Ec) + 31) & ~31;
+    int tabs = 2 * Er + 2 * Er + Er + 3 * Ec + Er + Ec;   // rin, rout (int64), rtab, ctab, cin, cout, signs
+    if (Ec % in.group == 0) tabs += Er * (Ec / in.group);  // scales of a codes tile
+    if (L.coef_single) {
+        // tensor-core build: both buffers hold index tables only; one
+        // coefficient area (128-byte aligned) is refilled stage by stage
+        L.coef_floats = (in.L ? stage_ucoef_floats(in.L, iL, jL, Er) : 0) + stage_ucoef_floats(in.R, iR, jR, Ec);
+        L.tab_base = 0;
+        L.buf_floats = (tabs + 3) & ~3;
+        L.coef_base = (L.tile_floats + 2 * L.buf_floats + 31) & ~31;
+        L.stage_base = L.coef_base + L.coef_floats;
+    } else {
+        L.coef_floats = (in.L ? stage_coef_floats(in.L, iL, jL, Er) : 0) + stage_coef_floats(in.R, iR, jR, Ec);
+        L.tab_base = (L.coef_floats + 1) & ~1;
+        L.buf_floats = (L.tab_base + tabs + 3) & ~3;
+        L.coef_base = 0;
+        L.stage_base = L.tile_floats + 2 * L.buf_floats;
+    }
     L.loc_base = L.stage_base + Er * Ec;                  // staging: fp32 tile (the largest input form)
     L.lev_base = L.loc_base + ((Er + Ec + 3) & ~3);
-    L.total_floats = L.lev_base + 32;
+    L.tc_base = L.lev_base + 32;                          // TMEM address slot, then 8-byte mbarriers
+    L.total_floats = L.tc_base + 2 + 2 * (2 * MAX_SLOTS_HOST + MAXPS + 1) + 2;
     return L;
 }
 
@@ -1156,6 +1594,7 @@ void fill_stages(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inve
     }
     D.nst = n;
     coef_floats = 0;
+    int ucoef_floats = 0;
     for (int u = 0; u < n; ++u) {
         const PlanDev *pl = refs[u].axis == 0 ? in.L : in.R;
         const int t = refs[u].t;
@@ -1178,6 +1617,17 @@ void fill_stages(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inve
         S.coef = inverse ? sd.pinv : sd.pfwd;
         S.had = stage_is_fwht(sd) ? 1 : 0;
         if (!S.had) coef_floats += S.G * S.gstride;
+        // tensor-core fields (used by the tcgen05 build)
+        const int NV = refs[u].axis == 0 ? D.ax[1].E : D.ax[0].E;
+        S.up = sd.up;
+        S.mb = NV >= 128 ? 128 : 64;
+        S.nvb = (NV + S.mb - 1) / S.mb;
+        S.nslots = 512 / (4 * sd.up);
+        S.ucoef = inverse ? sd.uinv : sd.ufwd;
+        S.ucoff = 4 * ucoef_floats;
+        S.f_nvb = make_fdiv(static_cast<unsigned>(S.nvb));
+        S.f_sig = make_fdiv(static_cast<unsigned>(S.sig));
+        if (!S.had) ucoef_floats += S.G * 2 * sd.up * sd.up;
     }
 }
 
@@ -1199,12 +1649,17 @@ int launch_pass_t(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
     const int64_t nb = D.ax[0].nt * D.ax[1].nt;
     if (nb <= 0) return 0;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(nb, nsm[dev]));
-    pass_kernel<PRO, EPI, SS><<<grid, PT, D.smem_bytes, st>>>(D, Q);
+    // The tensor-core build takes all 512 TMEM columns of its SM: asking for
+    // more than half of the SM's shared memory keeps it to one CTA per SM, so
+    // no second CTA ever waits on the allocation.
+    const int smem = (SS == SS_TC) ? std::max(D.smem_bytes, TC_MIN_SMEM) : D.smem_bytes;
+    pass_kernel<PRO, EPI, SS><<<grid, PT, smem, st>>>(D, Q);
     return cudaGetLastError();
 }
 
 template <int PRO, int EPI>
 int launch_pass(const PassDesc &D, const QuantDev &Q, cudaStream_t st) {
+    if (D.coef_single) return launch_pass_t<PRO, EPI, SS_TC>(D, Q, st);
     bool had = false, k16 = true;
     for (int u = 0; u < D.nst; ++u) {
         had = had || D.st[u].had;
@@ -1241,7 +1696,9 @@ void build_desc(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inver
     D.TCp = tcp_of(D.ax[1].E);
     const SmemLayout L = smem_layout(in, ps.iL, ps.jL, ps.iR, ps.jR, D.ax[0].E, D.ax[1].E);
     D.tile_floats = L.tile_floats;
-    D.coef_base = 0;
+    D.coef_base = L.coef_base;
+    D.coef_single = L.coef_single;
+    D.tc_base = L.tc_base;
     D.coef_floats = cf;
     D.tab_base = L.tab_base;
     D.buf_floats = L.buf_floats;
@@ -1269,6 +1726,19 @@ void record_event(int k, cudaStream_t st) {
 }
 
 }  // namespace
+
+void set_block_stages(int mode) { g_block_stage_mode = mode; }
+
+int pass_fault_status(unsigned *flags) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_pass_fault, sizeof(v));
+    if (e == cudaSuccess && v) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_pass_fault, &zero, sizeof(zero));
+    }
+    *flags = v;
+    return e;
+}
 
 void set_pass_events(void *const *events, int n) {
     t_events = (n > 0) ? events : nullptr;
@@ -1328,6 +1798,32 @@ void link_passes(PassDesc &D, const PlanInput &in, const std::vector<PassSpec> &
     }
 }
 
+// Whether the tensor-core build can fetch each tile's input with bulk
+// copies: the whole tile at once from a workspace in this pass's tile-major
+// order, or one copy per tile row when the tile's columns are contiguous and
+// every row's run starts and ends on a 16-byte boundary.
+void set_bulk_input(PassDesc &D, int pro, int bits, const void *src) {
+    D.in_bulk = 0;
+    D.in_row_bytes = 0;
+    if (!D.coef_single) return;
+    if (pro == PRO_F32) {
+        if (D.in_blocked) D.in_bulk = 1;
+        return;
+    }
+    const int Ec = D.ax[1].E;
+    for (int i = 0; i < Ec; ++i)
+        if (axis_global(D.ax[1], 0u, i) != axis_global(D.ax[1], 0u, 0) + i) return;
+    if (reinterpret_cast<uintptr_t>(src) % 16) return;
+    if (pro == PRO_BF16) {
+        if ((Ec * 2) % 16 || (D.ld_in * 2) % 16) return;
+        D.in_row_bytes = Ec * 2;
+    } else {
+        if ((Ec * bits) % 128 || (D.cols * bits / 8) % 16) return;
+        D.in_row_bytes = Ec * bits / 8;
+    }
+    D.in_bulk = 2;
+}
+
 }  // namespace
 
 int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q, const void *in_ptr,
@@ -1346,6 +1842,7 @@ int launch_pass_fwd(const PlanDev &left, const PlanDev &right, const QuantDev &q
         link_passes(D, in, ps, k, false, ws, in_ptr, nullptr);
         int pro = PRO_F32, epi = EPI_F32;
         if (first) pro = (in_dtype == HARP_BF16) ? PRO_BF16 : PRO_F32;
+        set_bulk_input(D, pro, q.bits, D.in);
         if (last) {
             epi = rotated_out ? EPI_QUANT_F32 : EPI_QUANT;
             D.bins = bins_exact(q, 64) ? 1 : 0;
@@ -1380,6 +1877,7 @@ int launch_pass_inv(const PlanDev &left, const PlanDev &right, const QuantDev &q
             D.in_codes = codes;
             D.in_scales = scales;
         }
+        set_bulk_input(D, pro, q.bits, first ? static_cast<const void *>(codes) : D.in);
         if (last) epi = (out_dtype == HARP_BF16) ? EPI_BF16 : EPI_F32;
         const int e = dispatch(D, q, pro, epi, st);
         if (e) return e;

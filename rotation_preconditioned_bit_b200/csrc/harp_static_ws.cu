@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "harp.h"
+#include "harp_internal.h"
 
 namespace {
 
@@ -61,8 +62,11 @@ int harp_rotate_quantize_static(harp_plan_t left, harp_plan_t right, harp_codebo
                                 uint8_t *codes, uint16_t *scales, float *rotated_out,
                                 void *stream) {
     if (!right || !cb) return HARP_ERR_INVALID_ARG;
+    // the plans must belong to the current device before its scratch array is picked
+    int st = harp::plans_on_current_device(left, right);
+    if (st) return st;
     size_t need = 0;
-    int st = harp_workspace_size(left, right, rows, cols, &need);
+    st = harp_workspace_size(left, right, rows, cols, &need);
     if (st) return st;
     if (need > kScratchBytes) return HARP_ERR_WORKSPACE;
     void *ws = nullptr;

@@ -18,7 +18,7 @@
 // No row exchange is needed: the symmetric part of I - A is the identity, so
 // every Schur complement met during elimination has a symmetric part >= I
 // and every pivot is >= 1 (no zero or tiny pivot, no growth).
-// The finished block goes to any of five layouts at once, so a plan's four
+// The finished block goes to any of seven layouts at once, so a plan's six
 // device copies of a stage are refreshed by one launch.
 #include <cuda_runtime.h>
 
@@ -100,6 +100,23 @@ theta_blocks_kernel(int b, int64_t n_groups, const int8_t *__restrict__ theta, d
             if (o.inv) o.inv[(c * b + k) * o.kpad + j] = v;
             if (o.pfwd) o.pfwd[(c * o.jp + j) * o.kp + k] = v;
             if (o.pinv) o.pinv[(c * o.jp + k) * o.kp + j] = v;
+            if (o.ufwd || o.uinv) {
+                // tensor-core operands: tf32-rounded coefficient and remainder
+                uint32_t hb, lb;
+                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hb) : "f"(v));
+                const float hi = __uint_as_float(hb);
+                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lb) : "f"(v - hi));
+                const float lo = __uint_as_float(lb);
+                const int64_t ub = c * 2 * o.up * o.up;
+                if (o.ufwd) {
+                    o.ufwd[ub + umma_block_index(k, j, o.up)] = hi;
+                    o.ufwd[ub + umma_block_index(o.up + k, j, o.up)] = lo;
+                }
+                if (o.uinv) {
+                    o.uinv[ub + umma_block_index(j, k, o.up)] = hi;
+                    o.uinv[ub + umma_block_index(o.up + j, k, o.up)] = lo;
+                }
+            }
         }
     }
 }

@@ -2,9 +2,9 @@
 
 Every input comes from the seeded generator (synth); the oracle builds its own
 float64 blocks and codebook from the same raw draws. Full-size workloads are
-compared element by element where the oracle finishes in seconds (the
-64x256, 4096x4096 and [T, 4096] workloads) and on sampled rows otherwise
-(4096x11008, 8192x28672), in the launch configuration the benchmark times.
+compared element by element, forward and inverse, at every full size (the
+oracle spreads its independent rows and columns over the host threads), in
+the launch configuration the benchmark times.
 """
 
 import numpy as np
@@ -39,11 +39,6 @@ def to_dev(w):
 
 def scales_np(t):
     return t.cpu().numpy().view(np.uint16)
-
-
-def sample_rows(rows, n, seed):
-    pick = synth.choose(seed, 77, rows, n - 3)
-    return np.unique(np.concatenate([[0, rows // 2, rows - 1], pick])).astype(np.int64)
 
 
 # ------------------------------------------------------------ 64 x 256 fp32, (16,16) Sylvester
@@ -101,6 +96,36 @@ def test_c2_two_sided_full_matrix(c2_ref, qi):
     assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
 
 
+@pytest.fixture(params=["tc", "ffma"])
+def block_stages(request):
+    """Run a test with the two-sided calls' block stages forced to the tensor
+    cores (tcgen05 3xTF32) or to fp32 FMAs; back to automatic afterwards."""
+    mode = harp.HARP_BLOCK_STAGES_TC if request.param == "tc" else harp.HARP_BLOCK_STAGES_FFMA
+    harp.harp_set_block_stages(mode)
+    yield request.param
+    harp.harp_set_block_stages(harp.HARP_BLOCK_STAGES_AUTO)
+
+
+def test_c2_both_block_stage_kinds_match_oracle(c2_ref, block_stages):
+    """The 4096 x 4096 workload through each block-stage implementation:
+    forward (2- and 4-bit Lloyd-Max, rotated copy and codes) and the inverse
+    of the oracle's own codes, every element against the oracle."""
+    w, ref = c2_ref
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    x = to_dev(w)
+    for q in w.quants:
+        oc, osc, m, sm = oracle.quantize(q.kind, q.bits, q.group, ref)
+        cb = harp.Codebook(q.kind, q.bits, q.group)
+        codes, scales, rot = harp.rotate_quantize(left, right, cb, x, want_rotated=True)
+        e = rel_l2(rot.cpu().numpy(), ref)
+        del rot
+        rep = compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, q.bits, q.group)
+        print(f"\nc2 {block_stages} {q.bits}-bit: rotated rel_l2 {e:.3e}", rep)
+        assert e <= TOL_F32
+        _inverse_full(w, left, right, q, oracle.pack(q.bits, oc), osc, Pl, Pr, f"c2 {block_stages} {q.bits}-bit")
+
+
 def test_c2_unfused_matches_oracle_like_fused(c2_ref):
     """The separate calls (left rotation, right rotation, standalone
     quantizer) meet the same bar against the oracle as the fused call. The
@@ -144,54 +169,75 @@ def test_c3_activation_rows(T):
     assert rel_l2(xb.float().cpu().numpy(), ref) <= TOL_BF16
 
 
-# ------------------------------------------------------------ sampled rows of the large workloads
+# ------------------------------------------------------------ inverse paths, whole matrices
 
-def _sampled_forward(w, q, which):
+def _inverse_full(w, left, right, q, raw, sc, Pl, Pr, label):
+    """dequantize + unrotate of the packed code stream `raw` with fp16 scales
+    `sc` (never produced by the CUDA path) against the oracle, every element,
+    fp32 and bf16 outputs."""
+    rows, cols = w.rows, w.cols
+    ref = oracle.dequantize_unrotate(oracle.unpack(q.bits, raw, cols), sc, Pl, Pr, q.kind, q.bits, q.group)
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    codes = torch.from_numpy(np.ascontiguousarray(raw)).cuda()
+    scales = torch.from_numpy(np.ascontiguousarray(sc).view(np.int16)).cuda()
+    out = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.float32)
+    e32 = rel_l2(out.cpu().numpy(), ref)
+    del out
+    outb = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.bfloat16)
+    e16 = rel_l2(outb.float().cpu().numpy(), ref)
+    print(f"\n{label}: inverse rel_l2 fp32 {e32:.3e} bf16 {e16:.3e}")
+    assert e32 <= TOL_F32
+    assert e16 <= TOL_BF16
+    return ref
+
+
+@pytest.mark.parametrize("qi", [0, 1])
+def test_c2_inverse_full_matrix(c2_ref, qi):
+    """The benchmarked inverse: 4096 x 4096, (16,16,16) on both sides,
+    2- and 4-bit Lloyd-Max g128, fp32 and bf16 outputs, every element --
+    on a seeded random code stream and on the oracle forward's own codes
+    (HARP section 5: the rotation is undone exactly by the transposes;
+    PolarQuant section 2: dequantise, then rotate back)."""
+    w, ref = c2_ref
+    q = w.quants[qi]
     Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
-    X = synth.x_as_f64(w)
-    ref = oracle.two_sided_rows(X, Pl, Pr, which)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    raw, sc = synth.random_code_stream(2020 + qi, w.rows, w.cols, q.bits, q.group)
+    _inverse_full(w, left, right, q, raw, sc, Pl, Pr, f"c2 {q.bits}-bit random stream")
+    oc, osc, _, _ = oracle.quantize(q.kind, q.bits, q.group, ref, with_margins=False)
+    _inverse_full(w, left, right, q, oracle.pack(q.bits, oc), osc, Pl, Pr, f"c2 {q.bits}-bit oracle codes")
+
+
+# ------------------------------------------------------------ the large workloads, whole matrices
+
+@pytest.fixture(scope="module")
+def c4_ref():
+    w = wl("c4")
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    return w, Pl, Pr, Pr.rotate_rows(Pl.rotate_cols(synth.x_as_f64(w)))
+
+
+def _full_forward(w, Pl, Pr, ref, q, label):
     oc, osc, m, sm = oracle.quantize(q.kind, q.bits, q.group, ref)
     left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
     cb = harp.Codebook(q.kind, q.bits, q.group)
     x = to_dev(w)
     codes, scales, rot = harp.rotate_quantize(left, right, cb, x, want_rotated=True)
-    idx = torch.from_numpy(which).cuda()
-    assert rel_l2(rot[idx].cpu().numpy(), ref) <= TOL_F32
-    rep = compare_quant(codes[idx].cpu().numpy(), scales_np(scales[idx]), oc, osc, m, sm, q.bits, q.group)
+    e = rel_l2(rot.cpu().numpy(), ref)
+    del rot
+    rep = compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, q.bits, q.group)
+    print(f"\n{label}: rotated rel_l2 {e:.3e}", rep)
+    assert e <= TOL_F32
+    # the benchmark's call (no fp32 copy) gives the same bytes
     codes2, scales2, _ = harp.rotate_quantize(left, right, cb, x)
     assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
-    return left, right, cb, codes, scales, rep
+    return left, right, cb, codes, scales, oc, osc
 
 
-def _sampled_inverse(w, q, which, seed):
-    """Random packed bytes and scales (any byte string is a valid code
-    stream) through dequantize + inverse rotation, against the oracle."""
-    rows, cols = w.rows, w.cols
-    raw, sc = synth.random_code_stream(seed, rows, cols, q.bits, q.group)
-    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
-    Wp = oracle.dequantize(q.kind, q.bits, q.group, oracle.unpack(q.bits, raw, cols), sc)
-    ref = oracle.inverse_rows(Wp, Pl, Pr, which)
-    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
-    cb = harp.Codebook(q.kind, q.bits, q.group)
-    codes = torch.from_numpy(raw).cuda()
-    scales = torch.from_numpy(sc.view(np.int16)).cuda()
-    out = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.float32)
-    idx = torch.from_numpy(which).cuda()
-    assert rel_l2(out[idx].cpu().numpy(), ref) <= TOL_F32
-    outb = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.bfloat16)
-    assert rel_l2(outb[idx].float().cpu().numpy(), ref) <= TOL_BF16
-    # standalone dequantise of the same bytes
-    deq = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
-    harp.harp_dequantize(cb, codes, scales, deq)
-    np.testing.assert_allclose(deq[idx].cpu().numpy(), Wp[which], rtol=0, atol=1e-6 * np.abs(Wp).max())
-
-
-def test_c4_forward_sampled_and_round_trip():
-    w = wl("c4")
+def test_c4_forward_full_and_round_trip(c4_ref):
+    w, Pl, Pr, ref = c4_ref
     q = w.quants[0]
-    which = sample_rows(w.rows, 12, 41)
-    left, right, cb, codes, scales, rep = _sampled_forward(w, q, which)
-    print("\nc4 3-bit:", rep)
+    left, right, cb, codes, scales, oc, osc = _full_forward(w, Pl, Pr, ref, q, "c4 3-bit")
     # round trip: an exact change of basis keeps the error norm
     What = harp.dequantize_unrotate(left, right, cb, codes, scales, w.rows, w.cols, torch.float32)
     Wp_hat = torch.empty((w.rows, w.cols), dtype=torch.float32, device="cuda")
@@ -201,26 +247,47 @@ def test_c4_forward_sampled_and_round_trip():
     e_orig = torch.linalg.norm((x - What).double()).item()
     e_rot = torch.linalg.norm((rot - Wp_hat).double()).item()
     assert abs(e_orig - e_rot) <= 1e-5 * e_rot
+    # the inverse of the oracle's own codes, every element
+    _inverse_full(w, left, right, q, oracle.pack(q.bits, oc), osc, Pl, Pr, "c4 3-bit oracle codes")
 
 
-def test_c4_inverse_sampled():
+def test_c4_inverse_full():
     w = wl("c4")
-    _sampled_inverse(w, w.quants[0], sample_rows(w.rows, 10, 43), 4040)
+    q = w.quants[0]
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    raw, sc = synth.random_code_stream(4040, w.rows, w.cols, q.bits, q.group)
+    _inverse_full(w, left, right, q, raw, sc, Pl, Pr, "c4 3-bit random stream")
+    # the standalone dequantiser on the same bytes
+    cb = harp.Codebook(q.kind, q.bits, q.group)
+    Wp = oracle.dequantize(q.kind, q.bits, q.group, oracle.unpack(q.bits, raw, w.cols), sc)
+    deq = torch.empty((w.rows, w.cols), dtype=torch.float32, device="cuda")
+    harp.harp_dequantize(cb, torch.from_numpy(raw).cuda(), torch.from_numpy(sc.view(np.int16)).cuda(), deq)
+    np.testing.assert_allclose(deq.cpu().numpy(), Wp, rtol=0, atol=1e-6 * np.abs(Wp).max())
+
+
+@pytest.fixture(scope="module")
+def c5_ref():
+    w = wl("c5")
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    return w, Pl, Pr, Pr.rotate_rows(Pl.rotate_cols(synth.x_as_f64(w)))
 
 
 @pytest.mark.parametrize("qi", [0, 1])
-def test_c5_forward_sampled(qi):
+def test_c5_forward_full(c5_ref, qi):
+    w, Pl, Pr, ref = c5_ref
+    q = w.quants[qi]
+    _full_forward(w, Pl, Pr, ref, q, f"c5 {q.kind} {q.bits}-bit")
+
+
+@pytest.mark.parametrize("qi", [0, 1])
+def test_c5_inverse_full(qi):
     w = wl("c5")
     q = w.quants[qi]
-    which = sample_rows(w.rows, 8, 51 + qi)
-    rep = _sampled_forward(w, q, which)[-1]
-    print(f"\nc5 {q.kind} {q.bits}-bit:", rep)
-
-
-@pytest.mark.parametrize("qi", [0, 1])
-def test_c5_inverse_sampled(qi):
-    w = wl("c5")
-    _sampled_inverse(w, w.quants[qi], sample_rows(w.rows, 6, 61 + qi), 5050 + qi)
+    Pl, Pr = oracle.processor(w.left), oracle.processor(w.right)
+    left, right = harp.Plan.from_side(w.left), harp.Plan.from_side(w.right)
+    raw, sc = synth.random_code_stream(5050 + qi, w.rows, w.cols, q.bits, q.group)
+    _inverse_full(w, left, right, q, raw, sc, Pl, Pr, f"c5 {q.kind} {q.bits}-bit random stream")
 
 
 # ------------------------------------------------------------ small shapes, every radix path
@@ -326,6 +393,31 @@ def test_plan_info_and_workspace():
     assert harp.workspace_size(None, plan, 7, 11008) == 0
 
 
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2,
+                    reason="needs a second device to make the current one differ from the plan's")
+def test_calls_refuse_a_plan_of_another_device():
+    """A plan's blocks live on the device that was current at creation; every
+    launching call made with another device current returns
+    HARP_ERR_INVALID_ARG before touching memory."""
+    torch.cuda.set_device(0)
+    s16 = synth.side_draws(1, (16, 16), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    plan = harp.Plan.from_side(s16)
+    cb = harp.Codebook("lloyd_max", 4, 128)
+    try:
+        torch.cuda.set_device(1)
+        st = harp.lib().harp_rotate(plan.handle, harp.HARP_RIGHT, harp.HARP_FWD, None, harp.HARP_F32,
+                                    None, harp.HARP_F32, 4, 256, 256, 256, None)
+        assert st == 1
+        st = harp.lib().harp_rotate_quantize(None, plan.handle, cb.handle, None, harp.HARP_F32, 4, 256,
+                                             None, None, None, None, 0, None)
+        assert st == 1
+        st = harp.lib().harp_rotate_quantize_static(plan.handle, plan.handle, cb.handle, None,
+                                                    harp.HARP_F32, 256, 256, None, None, None, None)
+        assert st == 1
+    finally:
+        torch.cuda.set_device(0)
+
+
 def test_pass_events_time_each_pass():
     """harp_pass_count reports the pass kernels of the two-sided calls and
     harp_set_pass_events gets one event per pass boundary recorded; results
@@ -380,7 +472,7 @@ def test_hadamard_two_sided_matches_oracle():
     assert rel_l2(out.cpu().numpy(), ref3) <= TOL_F32
 
 
-def test_mixed_radix_5120_two_sided():
+def test_mixed_radix_5120_two_sided(block_stages):
     """HARP section 2.1's arbitrary-d example, 5120 = 8 * 8 * 8 * 5 * 2, as
     the column processor of a 5120 x 1280 weight (row processor (5, 16, 16)),
     random orthogonal blocks: the fused forward with 3-bit Lloyd-Max g128 and
@@ -398,8 +490,15 @@ def test_mixed_radix_5120_two_sided():
     codes, scales, rot = harp.rotate_quantize(left, right, cb, xb, want_rotated=True)
     assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
     compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, 3, 128)
-    ref_inv = oracle.dequantize_unrotate(np_unpack(codes.cpu().numpy(), 3, cols), scales_np(scales),
-                                         Pl, Pr, "lloyd_max", 3, 128)
-    out = harp.dequantize_unrotate(left, right, cb, codes, scales, rows, cols, torch.float32)
+    # the inverse of the oracle's own codes (no oracle input comes from the CUDA path)
+    ref_inv = oracle.dequantize_unrotate(oc, osc, Pl, Pr, "lloyd_max", 3, 128)
+    out = harp.dequantize_unrotate(left, right, cb, torch.from_numpy(oracle.pack(3, oc)).cuda(),
+                                   torch.from_numpy(osc.view(np.int16)).cuda(), rows, cols, torch.float32)
     assert rel_l2(out.cpu().numpy(), ref_inv) <= TOL_F32
 
+
+
+def test_no_kernel_wait_ran_out():
+    """Every wait inside the library's kernels is bounded and records when it
+    runs out; none did during the tests above."""
+    assert harp.harp_fault_status() == 0

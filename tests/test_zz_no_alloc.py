@@ -11,8 +11,6 @@ matrix whose intermediate exceeds the array is refused before any launch.
 This file is named so that pytest collects it last.
 """
 
-import ctypes
-
 import numpy as np
 import pytest
 
@@ -25,6 +23,7 @@ pytestmark = pytest.mark.gpu
 
 def _case(rows_radix, cols_radix, bits, group, seed):
     import torch
+    torch.cuda.set_device(0)
     left_s = synth.side_draws(seed, rows_radix, "qr", synth.S_SIGNS_L, synth.S_BLOCKS_L)
     right_s = synth.side_draws(seed, cols_radix, "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
     rows, cols = int(np.prod(rows_radix)), int(np.prod(cols_radix))
@@ -61,14 +60,34 @@ def test_static_workspace_matches_caller_workspace_twice():
         assert rel_l2(rot.cpu().numpy(), ref_rot) <= TOL_F32
 
 
-def test_static_workspace_rejects_oversized_matrix():
+def test_static_workspace_five_bit_codes_match_twice():
+    """5-bit (PolarQuant Q5) codes take the whole-vector kernels, which write
+    the same library array through another path: two calls in a row match
+    the caller-workspace call."""
     import torch
-    torch.cuda.set_device(0)
-    # 4096 x 4096 needs a 128 MiB workspace: refused before any pointer is used
+    left, right, cb, x = _case((16, 8, 8), (8, 8, 16), 5, 128, 41)
+    rows, cols = x.shape
+    assert harp.workspace_size(left, right, rows, cols) <= harp.HARP_STATIC_WORKSPACE_BYTES
+    ref_codes, ref_scales = harp.empty_codes(rows, cols, cb)
+    ws = harp.empty_workspace(left, right, rows, cols)
+    harp.harp_rotate_quantize(left, right, cb, x, ref_codes, ref_scales, None, ws)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        codes, scales = harp.empty_codes(rows, cols, cb)
+        codes.fill_(0x5A)
+        harp.harp_rotate_quantize_static(left, right, cb, x, codes, scales, None)
+        torch.cuda.synchronize()
+        assert torch.equal(codes.cpu(), ref_codes.cpu())
+        assert torch.equal(scales.cpu(), ref_scales.cpu())
+
+
+def test_static_workspace_rejects_oversized_matrix():
+    # 4096 x 4096 needs a 128 MiB workspace: refused before any pointer is
+    # used. The data pointers are NULL, so a reordering of the checks would
+    # surface as HARP_ERR_INVALID_ARG, never as a launch.
     left, right, cb, _ = _case((16, 16, 16), (16, 16, 16), 2, 128, 5)
     assert harp.workspace_size(left, right, 4096, 4096) > harp.HARP_STATIC_WORKSPACE_BYTES
-    dummy = ctypes.c_void_p(1 << 20)
-    st = harp.lib().harp_rotate_quantize_static(left.handle, right.handle, cb.handle, dummy,
-                                                harp.HARP_BF16, 4096, 4096, dummy, dummy, None,
+    st = harp.lib().harp_rotate_quantize_static(left.handle, right.handle, cb.handle, None,
+                                                harp.HARP_BF16, 4096, 4096, None, None, None,
                                                 None)
     assert st == 5  # HARP_ERR_WORKSPACE
