@@ -270,6 +270,40 @@ def run_gpu(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
 
+    # ---- the same step with every block stage forced onto the tensor cores
+    # (tcgen05, 3xTF32), timed the same way, for comparison with the
+    # automatic choice above (every rank takes the same steps)
+    alt = None
+    if not args.no_alt:
+        harp.harp_set_block_stages(harp.HARP_BLOCK_STAGES_TC)
+        kt_tc = {k: [] for k in kt}
+        for _ in range(args.warmup):
+            flush.zero_()
+            step(False)
+        for _ in range(2 * len(BITS) * args.steps):
+            ev_pool.append(new_events(npass + 1))
+        torch.cuda.synchronize()
+        alt_ms, alt_evs = [], []
+        for _ in range(args.steps):
+            flush.zero_()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            evs = step(True)
+            s1.record(stream)
+            alt_evs.append((s0, s1, evs))
+        torch.cuda.synchronize()
+        harp.harp_set_block_stages(harp.HARP_BLOCK_STAGES_AUTO)
+        for s0, s1, evs in alt_evs:
+            alt_ms.append(s0.elapsed_time(s1))
+            for bits, ef, ei in evs:
+                for k in range(npass):
+                    kt_tc[f"fwd_p{k}_{bits}bit"].append(ef[k].elapsed_time(ef[k + 1]))
+                    kt_tc[f"inv_p{k}_{bits}bit"].append(ei[k].elapsed_time(ei[k + 1]))
+        alt = (max_over_ranks(sum(alt_ms), world, dev), kt_tc)
+        if world > 1:
+            torch.distributed.barrier()
+
     # ---- end to end through the public two-sided calls, host buffers
     e2e = None
     if not args.no_e2e:
@@ -325,7 +359,7 @@ def run_gpu(args, rank, world, local_rank):
                       "device-to-host copies on a second stream overlapping the next call",
                "workspace_bytes": ws_bytes}
     del flush
-    return total_ms, step_ms, kt, clk, e2e, npass, pass_fma
+    return total_ms, step_ms, kt, clk, e2e, npass, pass_fma, alt
 
 
 WORKLOAD_NAMES = ("c1", "c3", "c4", "c5", "rht", "pq", "theta")
@@ -356,7 +390,12 @@ def run_workloads(steps, dev, names=WORKLOAD_NAMES):
         return a.elapsed_time(b) / steps * 1e-3
 
     out = {}
+    jobs = []
     for name in [n for n in ("c1", "c3", "c4", "c5", "rht") if n in names]:
+        # the activation workload at every token count (T <= 16 is a
+        # latency case: its time in microseconds is the figure to read)
+        jobs += [(name, T) for T in (1, 16, 256, 8192)] if name == "c3" else [(name, None)]
+    for name, tokens in jobs:
         if name == "rht":
             # the c2 weight with Hadamard-initialised processors on both sides
             # (random signs, normalised Sylvester blocks: HARP's theta = 0 start)
@@ -365,6 +404,8 @@ def run_workloads(steps, dev, names=WORKLOAD_NAMES):
                            right=synth.side_draws(2, RADIX, "hadamard", synth.S_SIGNS_R, synth.S_BLOCKS_R),
                            left=synth.side_draws(2, RADIX, "hadamard", synth.S_SIGNS_L, synth.S_BLOCKS_L),
                            quants=[synth.Quant("lloyd_max", 4, GROUP)])
+        elif tokens is not None:
+            w = synth.workload(name, tokens=tokens)
         else:
             w = synth.workload(name)
         rows, cols = w.rows, w.cols
@@ -517,44 +558,48 @@ def _c2_oracle_inputs():
 
 
 def oracle_sample(frac):
-    """The float64 oracle on a sample of the step: the left pass on a column
-    strip and the right pass + quantise + inverse on a row strip, each a
-    fraction `frac` of the weight, for the 2-bit variant. Returns (seconds,
+    """The float64 oracle on a sample of the step, for each bit width of the
+    step: the left pass on a column strip and the right pass + quantise +
+    pack + dequantise + inverse on a row strip, each a fraction `frac` of the
+    weight, with the oracle's current host threads. Returns (seconds,
     algorithmic bytes credited, description)."""
     import oracle
 
     X, (Pl, Pr) = _c2_oracle_inputs()
     nc = max(1, int(round(COLS * frac)))
     nr = max(1, int(round(ROWS * frac)))
-    bits = BITS[0]
     t0 = time.perf_counter()
-    T = Pl.rotate_cols(X[:, :nc])
-    Y = Pr.rotate_rows(X[:nr, :])
-    codes, scales, _, _ = oracle.quantize("lloyd_max", bits, GROUP, Y, with_margins=False)
-    packed = oracle.pack(bits, codes)
-    codes2 = oracle.unpack(bits, packed, COLS)
-    Yh = oracle.dequantize("lloyd_max", bits, GROUP, codes2, scales)
-    Z = Pr.rotate_rows(Yh, inverse=True)
-    U = Pl.rotate_cols(T, inverse=True)
+    for bits in BITS:
+        T = Pl.rotate_cols(X[:, :nc])
+        Y = Pr.rotate_rows(X[:nr, :])
+        codes, scales, _, _ = oracle.quantize("lloyd_max", bits, GROUP, Y, with_margins=False)
+        packed = oracle.pack(bits, codes)
+        codes2 = oracle.unpack(bits, packed, COLS)
+        Yh = oracle.dequantize("lloyd_max", bits, GROUP, codes2, scales)
+        Z = Pr.rotate_rows(Yh, inverse=True)
+        U = Pl.rotate_cols(T, inverse=True)
+        del T, Z, U
     dt = time.perf_counter() - t0
-    del T, Z, U
     elems = nc * ROWS                              # both sides cover this many elements
-    credited = elems * (fwd_bytes_per_elem(bits) + inv_bytes_per_elem(bits))
-    desc = (f"float64 oracle, 2-bit variant: left pass on a {ROWS}x{nc} column strip and right pass "
-            f"+ quantise + pack + dequantise + inverse on a {nr}x{COLS} row strip "
-            f"({frac:.3f} of the weight), single thread")
+    credited = elems * sum(fwd_bytes_per_elem(b) + inv_bytes_per_elem(b) for b in BITS)
+    nt = oracle.threads()
+    desc = (f"float64 oracle, the step's {' and '.join(f'{b}-bit' for b in BITS)} variants: left pass on a "
+            f"{ROWS}x{nc} column strip and right pass + quantise + pack + dequantise + inverse on a "
+            f"{nr}x{COLS} row strip ({frac:.4f} of the weight), {nt} host thread{'s' if nt > 1 else ''}")
     return dt, credited, desc
 
 
 def pick_frac(budget_s):
-    dt, _, _ = oracle_sample(1.0 / 64)
-    per_full = dt * 64
-    return max(1.0 / 256, min(1.0, budget_s / per_full))
+    dt, _, _ = oracle_sample(1.0 / 128)
+    per_full = dt * 128
+    return max(1.0 / 512, min(1.0, budget_s / per_full))
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return
+    import oracle
+    cores = oracle.threads(os.cpu_count() or 1)
     budget = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     frac = pick_frac(budget)
     for _ in range(args.warmup):
@@ -571,7 +616,7 @@ def run_reference(args, world, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": WORKLOAD, "parallelism": "replicas", "l2": "n/a (host)"},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -588,6 +633,8 @@ def main():
     ap.add_argument("--impl", default="harp", choices=["harp", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-alt", action="store_true",
+                    help="skip the comparison series with every block stage on the tensor cores")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--workloads", action="store_true",
                     help="also time the c1, c3, c4 and c5 workloads (adds ~1 min of input generation)")
@@ -619,7 +666,7 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    total_ms, step_ms, kt, clk, e2e, npass, pass_fma = run_gpu(args, rank, world, local_rank)
+    total_ms, step_ms, kt, clk, e2e, npass, pass_fma, alt = run_gpu(args, rank, world, local_rank)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -639,10 +686,18 @@ def main():
                 "own_bytes_hbm_frac": round(d["own_gbs"] / hbm, 4)}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            frac = pick_frac(args.cpu_budget)
-            dt, credited, desc = oracle_sample(frac)
-            cpu = {"value": round(credited / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                   "sample": desc, "seconds": round(dt, 2)}
+            import oracle
+            cores = os.cpu_count() or 1
+            oracle.threads(1)
+            frac = pick_frac(args.cpu_budget / 2)
+            dt1, credited1, desc1 = oracle_sample(frac)
+            oracle.threads(cores)
+            frac_all = min(1.0, frac * cores)
+            dt, credited, desc = oracle_sample(frac_all)
+            cpu = {"value": round(credited / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+                   "sample": desc, "seconds": round(dt, 2),
+                   "single_thread": {"value": round(credited1 / dt1 / 1e9, 4), "cores": 1, "sample": desc1,
+                                     "seconds": round(dt1, 2)}}
         wl = (run_workloads(max(3, args.steps // 4), torch.device("cuda", local_rank))
               if args.workloads and world == 1 else None)
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -657,6 +712,23 @@ def main():
                 "hbm_frac": round(value / world / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": peak_src,
                 "roofline": roof, "kernels": ktab, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 2 * len(BITS) * npass * args.steps, "clocks": clk}
+        # the metric's own call, rotate + quantize alone: per bit width the
+        # forward passes' device time and the forward's algorithmic bytes
+        fwd = {}
+        for b in BITS:
+            us = sum(ktab[f"fwd_p{k}_{b}bit"]["us"] for k in range(npass))
+            gbs = ROWS * COLS * fwd_bytes_per_elem(b) / (us * 1e-6) / 1e9
+            fwd[f"{b}bit"] = {"us": round(us, 2), "gbs": round(gbs, 2), "hbm_frac": round(gbs / hbm, 4)}
+        line["forward_only"] = fwd
+        if alt is not None:
+            alt_ms, kt_tc = alt
+            ktab_tc = kernel_table(kt_tc, npass, pass_fma)
+            line["tensor_core_stages"] = {
+                "ms_per_step": round(alt_ms / args.steps, 4),
+                "value": round(job_gbs(world, args.steps, alt_ms), 2),
+                "note": "same step with every block stage on tcgen05 (kind::tf32, split operands); the "
+                        "headline uses the automatic choice (FFMA for 16-wide blocks)",
+                "kernels_us": {k: v["us"] for k, v in ktab_tc.items()}}
         if wl is not None:
             line["workloads"] = wl
         print(json.dumps(line), flush=True)

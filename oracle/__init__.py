@@ -78,6 +78,7 @@ def _set_types(L):
     L.orc_f16_value.argtypes = [ctypes.c_uint16]
     L.orc_f16_value.restype = ctypes.c_double
     L.orc_quantize.argtypes = [_INT, _INT, _L, _L, _L, _D, _U8, _U16, _D, _D]
+    L.orc_quantize_mode.argtypes = [_INT, _INT, _L, _INT, _L, _L, _D, _U8, _U16, _D, _D]
     L.orc_dequantize.argtypes = [_INT, _INT, _L, _L, _L, _U8, _U16, _D]
     L.orc_pack.argtypes = [_INT, _L, _L, _U8, _U8]
     L.orc_unpack.argtypes = [_INT, _L, _L, _U8, _U8]
@@ -238,15 +239,20 @@ def f16_value(h):
     return float(lib().orc_f16_value(int(h)))
 
 
-def quantize(kind, bits, group, X, with_margins=True):
+SCALE_MODES = {"rms": 0, "absmax": 1}
+
+
+def quantize(kind, bits, group, X, with_margins=True, scale_mode="rms"):
+    """Group-wise codes and fp16 scales of X; scale_mode 'rms' (default) or
+    'absmax' (Lloyd-Max only: s = max|x| / largest centroid)."""
     X = np.ascontiguousarray(X, dtype=np.float64)
     rows, cols = X.shape
     codes = np.empty((rows, cols), dtype=np.uint8)
     scales = np.empty((rows, cols // group), dtype=np.uint16)
     margin = np.empty((rows, cols), dtype=np.float64) if with_margins else None
     smargin = np.empty((rows, cols // group), dtype=np.float64) if with_margins else None
-    _chk(lib().orc_quantize(KINDS[kind], bits, group, rows, cols, _p(X, _D), _p(codes, _U8),
-                            _p(scales, _U16), _p(margin, _D), _p(smargin, _D)), "quantize")
+    _chk(lib().orc_quantize_mode(KINDS[kind], bits, group, SCALE_MODES[scale_mode], rows, cols, _p(X, _D),
+                                 _p(codes, _U8), _p(scales, _U16), _p(margin, _D), _p(smargin, _D)), "quantize")
     return codes, scales, margin, smargin
 
 

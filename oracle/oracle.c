@@ -574,11 +574,29 @@ static void orc_tables(int bits, const double *c64, float *cent, float *thr)
  *  margin[i] = distance of z = x/s to the nearest decision boundary;
  *  scale_margin[g] = |pre-rounding scale - nearest fp16 rounding midpoint|
  *                    relative to the scale (how close the fp16 decision was). */
+int orc_quantize_mode(int kind, int bits, int64_t group, int scale_mode, int64_t rows, int64_t cols,
+                      const double *X, uint8_t *codes, uint16_t *scales,
+                      double *margin, double *scale_margin);
+
 int orc_quantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
                  const double *X, uint8_t *codes, uint16_t *scales,
                  double *margin, double *scale_margin)
 {
+    return orc_quantize_mode(kind, bits, group, 0, rows, cols, X, codes, scales, margin, scale_margin);
+}
+
+/* As orc_quantize, with the Lloyd-Max group scale chosen by scale_mode:
+ *  0: s = sqrt(mean of squares) (the default reading of PolarQuant's
+ *     normalisation to N(0,1));
+ *  1: s = max|x| / c_{K-1}, the group's largest magnitude mapped onto the
+ *     outermost fp32 centroid (the alternative kept as a flag).
+ * Absmax codebooks accept mode 0 only. */
+int orc_quantize_mode(int kind, int bits, int64_t group, int scale_mode, int64_t rows, int64_t cols,
+                      const double *X, uint8_t *codes, uint16_t *scales,
+                      double *margin, double *scale_margin)
+{
     if (bits < 2 || bits > 5 || group <= 0 || cols % group) return ORC_BAD;
+    if (scale_mode < 0 || scale_mode > 1 || (kind != 0 && scale_mode != 0)) return ORC_BAD;
     int K = 1 << bits;
     int qmax = (1 << (bits - 1)) - 1;
     double c64[32];
@@ -593,7 +611,11 @@ int orc_quantize(int kind, int bits, int64_t group, int64_t rows, int64_t cols,
         for (int64_t g = 0; g < ng; ++g) {
             const double *x = X + r * cols + g * group;
             double s_exact;
-            if (kind == 0) {
+            if (kind == 0 && scale_mode == 1) {
+                double mx = 0.0;
+                for (int64_t i = 0; i < group; ++i) if (fabs(x[i]) > mx) mx = fabs(x[i]);
+                s_exact = mx / (double)cent[K - 1];
+            } else if (kind == 0) {
                 double ss = 0.0;
                 for (int64_t i = 0; i < group; ++i) ss += x[i] * x[i];
                 s_exact = sqrt(ss / (double)group);

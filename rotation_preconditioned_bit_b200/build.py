@@ -21,6 +21,7 @@ OBJDIR = os.path.join(HERE, "_build")
 SOURCES = [os.path.join(CSRC, f) for f in ("harp_kernels.cu", "harp_pass.cu", "harp_api.cpp", "harp_static_ws.cu",
                                               "harp_theta.cu", "harp_short.cu")]
 HEADERS = [os.path.join(CSRC, "harp_internal.h"), os.path.join(CSRC, "harp_quant_dev.cuh"),
+           os.path.join(CSRC, "harp_tc.cuh"),
            os.path.join(INCLUDE, "harp.h")]
 CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")

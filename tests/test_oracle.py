@@ -444,6 +444,39 @@ def test_lloyd_max_codes_are_nearest_centroid(bits, group):
     np.testing.assert_array_equal(scales, rms.astype(np.float16).view(np.uint16))
 
 
+@pytest.mark.parametrize("bits,group", [(2, 64), (3, 128), (4, 128), (5, 128)])
+def test_lloyd_max_absmax_scale_mode(bits, group):
+    """The alternative Lloyd-Max scale (largest magnitude onto the outermost
+    centroid): the stored scale is fp16(max|x| / c_{K-1}) computed with
+    numpy; codes are still the nearest centroid of x/s (brute force); the
+    group's largest-magnitude element gets an outermost code; the mode is
+    refused for absmax codebooks."""
+    X = synth.small_matrix(31 + bits, 12, 512, outlier_cols=3, scale=0.02)
+    codes, scales, margin, smargin = oracle.quantize("lloyd_max", bits, group, X, scale_mode="absmax")
+    c, _ = oracle.lloyd_max(bits)
+    cent = c.astype(np.float32).astype(np.float64)
+    K = 1 << bits
+    amax = np.abs(X.reshape(12, -1, group)).max(axis=2)
+    np.testing.assert_array_equal(scales, (amax / cent[-1]).astype(np.float16).view(np.uint16))
+    s = np.repeat(np.array([[oracle.f16_value(v) for v in row] for row in scales]), group, axis=1)
+    brute = _brute_nearest(X / s, cent)
+    safe = margin > 1e-9
+    assert np.mean(safe) > 0.999
+    np.testing.assert_array_equal(codes[safe], brute[safe])
+    Xg = X.reshape(12, -1, group)
+    cg = codes.reshape(12, -1, group)
+    im = np.argmax(np.abs(Xg), axis=2)
+    for r in range(12):
+        for g in range(Xg.shape[1]):
+            i = im[r, g]
+            assert cg[r, g, i] == (K - 1 if Xg[r, g, i] > 0 else 0)
+    # differs from the default RMS reading
+    codes0, scales0, _, _ = oracle.quantize("lloyd_max", bits, group, X)
+    assert not np.array_equal(scales, scales0)
+    with pytest.raises(ValueError):
+        oracle.quantize("absmax", bits, group, X, scale_mode="absmax")
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4, 5])
 def test_absmax_codes(bits):
     X = synth.small_matrix(21 + bits, 8, 256, outlier_cols=2)
