@@ -30,7 +30,8 @@
  *    (d = cols; X -> X V with V = M^T). HARP_LEFT maps every column w to M w
  *    (d = rows; W -> U^T W with U = M^T). Two-sided: W' = M_L W M_R^T.
  *  - Quantizer groups are `group` consecutive columns of a row of the rotated
- *    matrix. Lloyd-Max: s = sqrt(mean(x^2)) over the group; code = number of
+ *    matrix. Lloyd-Max: s = sqrt(mean(x^2)) over the group (or, with
+ *    HARP_SCALE_ABSMAX, max|x| / c_{K-1}); code = number of
  *    fp32 midpoints t_k (of neighbouring fp32 centroids) with x/s > t_k.
  *    Absmax: s = max|x| / (2^(b-1) - 1); code = clamp(rint(x/s), -qmax, qmax)
  *    + 2^(b-1), so 4-bit codes are 1..15. Scales are stored as IEEE fp16
@@ -110,11 +111,15 @@ int harp_version(void);
  *         exact inverses only if they are orthogonal.
  *  signs  host [d] of +1/-1 (any float is accepted and multiplied in), or
  *         NULL for all +1.
- * The plan copies blocks and signs to device memory (synchronously) and owns
- * that copy until harp_plan_destroy. Errors: INVALID_ARG (NULL out/radix/
- * blocks), UNSUPPORTED, SHAPE, CUDA, ALLOC. */
+ *  stream CUDA stream the copies to device memory are ordered on (NULL =
+ *         legacy default stream).
+ * The plan copies blocks and signs to device memory and owns that copy until
+ * harp_plan_destroy. The copies run on `stream` and are complete when the
+ * call returns (it synchronises that stream), so the caller may release its
+ * host arrays at once and launches on any stream may use the plan. Errors:
+ * INVALID_ARG (NULL out/radix/blocks), UNSUPPORTED, SHAPE, CUDA, ALLOC. */
 int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
-                     const float *const *blocks, const float *signs);
+                     const float *const *blocks, const float *signs, void *stream);
 
 /* Release a plan and its device memory. NULL is accepted. The caller must
  * ensure no launch that uses the plan is still running. */
@@ -192,16 +197,26 @@ int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float
 int harp_lloyd_max_centroids(int bits, float *out);
 
 /* Create a quantizer description  [PolarQuant 1, 2].
- *  kind       HARP_LLOYD_MAX or HARP_ABSMAX.
- *  bits       2, 3, 4 or 5 (PolarQuant section 3 uses 5-bit Q5 codes).
- *  group      elements per scale group along a row: a positive multiple of
- *             32 (UNSUPPORTED otherwise); must divide cols at each call
- *             (group = cols gives one scale per row).
- *  centroids  host [2^bits] ascending floats for HARP_LLOYD_MAX, or NULL for
- *             the built-in N(0,1) Lloyd-Max table; ignored for absmax.
+ *  kind        HARP_LLOYD_MAX or HARP_ABSMAX.
+ *  bits        2, 3, 4 or 5 (PolarQuant section 3 uses 5-bit Q5 codes).
+ *  group       elements per scale group along a row: a positive multiple of
+ *              32 (UNSUPPORTED otherwise); must divide cols at each call
+ *              (group = cols gives one scale per row).
+ *  scale_mode  how a Lloyd-Max group is scaled to N(0,1):
+ *              HARP_SCALE_RMS (default): s = sqrt(mean(x^2)) over the group
+ *              (PolarQuant section 2: l2-normalise, then scale to unit
+ *              variance); HARP_SCALE_ABSMAX: s = max|x| / c_{K-1}, the
+ *              group's largest magnitude onto the outermost centroid. Absmax
+ *              codebooks always use s = max|x| / (2^(b-1) - 1) and accept
+ *              either value.
+ *  centroids   host [2^bits] ascending floats for HARP_LLOYD_MAX, or NULL
+ *              for the built-in N(0,1) Lloyd-Max table; ignored for absmax.
  * Host-only object (no device memory); the tables travel as kernel arguments.
- * Errors: INVALID_ARG, UNSUPPORTED, ALLOC. */
-int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group,
+ * Errors: INVALID_ARG (NULL out, unknown kind or scale_mode, centroids not
+ * strictly ascending, or a non-positive largest centroid with
+ * HARP_SCALE_ABSMAX), UNSUPPORTED, ALLOC. */
+enum harp_scale_mode { HARP_SCALE_RMS = 0, HARP_SCALE_ABSMAX = 1 };
+int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group, int scale_mode,
                          const float *centroids);
 int harp_codebook_destroy(harp_codebook_t cb);
 

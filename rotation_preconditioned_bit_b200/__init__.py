@@ -68,13 +68,13 @@ def lib():
         L.harp_status_string.argtypes = [_INT]
         L.harp_plan_create.argtypes = [ctypes.POINTER(_P), _I64, _INT, ctypes.POINTER(ctypes.c_int32),
                                        ctypes.POINTER(ctypes.POINTER(ctypes.c_float)),
-                                       ctypes.POINTER(ctypes.c_float)]
+                                       ctypes.POINTER(ctypes.c_float), _P]
         L.harp_plan_destroy.argtypes = [_P]
         L.harp_plan_info.argtypes = [_P, ctypes.POINTER(_I64), ctypes.POINTER(_INT),
                                      ctypes.POINTER(ctypes.c_int32)]
         L.harp_stage_blocks.argtypes = [_INT, _INT, _I64, _P, _P, ctypes.c_double, _P]
         L.harp_lloyd_max_centroids.argtypes = [_INT, _P]
-        L.harp_codebook_create.argtypes = [ctypes.POINTER(_P), _INT, _INT, _I64, _P]
+        L.harp_codebook_create.argtypes = [ctypes.POINTER(_P), _INT, _INT, _I64, _INT, _P]
         L.harp_codebook_destroy.argtypes = [_P]
         L.harp_codebook_tables.argtypes = [_P, _P, _P]
         L.harp_workspace_size.argtypes = [_P, _P, _I64, _I64, ctypes.POINTER(ctypes.c_size_t)]
@@ -130,7 +130,7 @@ def lloyd_max_centroids(bits: int) -> np.ndarray:
 class Plan:
     """A processor plan (radix schedule, float32 blocks, signs) on the current device."""
 
-    def __init__(self, radix, blocks, signs=None):
+    def __init__(self, radix, blocks, signs=None, stream=None):
         radix = [int(b) for b in radix]
         self.radix = tuple(radix)
         self.d = int(np.prod(radix))
@@ -142,7 +142,8 @@ class Plan:
         h = _P()
         _check(lib().harp_plan_create(ctypes.byref(h), self.d, len(radix), rad, ptrs,
                                       None if self._signs is None else
-                                      self._signs.ctypes.data_as(ctypes.POINTER(ctypes.c_float))),
+                                      self._signs.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                      _stream(stream)),
                "harp_plan_create")
         self.handle = h
 
@@ -174,15 +175,20 @@ class Plan:
             pass
 
 
-class Codebook:
-    """Quantizer description: kind ('lloyd_max' | 'absmax'), bits, group."""
+SCALE_MODES = {"rms": 0, "absmax": 1}
 
-    def __init__(self, kind, bits, group, centroids=None):
+
+class Codebook:
+    """Quantizer description: kind ('lloyd_max' | 'absmax'), bits, group,
+    Lloyd-Max scale mode ('rms' default | 'absmax')."""
+
+    def __init__(self, kind, bits, group, centroids=None, scale_mode="rms"):
         self.kind = QUANT_KINDS.get(kind, kind)
         self.bits, self.group = int(bits), int(group)
+        self.scale_mode = SCALE_MODES.get(scale_mode, scale_mode)
         c = None if centroids is None else np.ascontiguousarray(centroids, dtype=np.float32)
         h = _P()
-        _check(lib().harp_codebook_create(ctypes.byref(h), self.kind, self.bits, self.group,
+        _check(lib().harp_codebook_create(ctypes.byref(h), self.kind, self.bits, self.group, self.scale_mode,
                                           None if c is None else c.ctypes.data), "harp_codebook_create")
         self.handle = h
 
@@ -226,6 +232,8 @@ def _dtype_code(t):
 def _stream(stream):
     import torch
     if stream is None:
+        if not torch.cuda.is_available():
+            return None            # the library reports the missing device itself
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
 

@@ -299,7 +299,7 @@ int harp_lloyd_max_centroids(int bits, float *out) {
 }
 
 int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
-                     const float *const *blocks, const float *signs) {
+                     const float *const *blocks, const float *signs, void *stream) {
     if (!out || !radix || !blocks) return HARP_ERR_INVALID_ARG;
     *out = nullptr;
     if (m < 1 || m > HARP_MAX_STAGES) return HARP_ERR_UNSUPPORTED;
@@ -387,7 +387,11 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
         delete p;
         return HARP_ERR_ALLOC;
     }
-    if (cudaMemcpy(p->mem, host.data(), total * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
+    // ordered on the caller's stream, finished before returning (the host
+    // staging copy and the caller's arrays may go away afterwards)
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(p->mem, host.data(), total * sizeof(float), cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaStreamSynchronize(cs) != cudaSuccess) {
         cudaGetLastError();
         cudaFree(p->mem);
         delete p;
@@ -476,11 +480,12 @@ int harp_plan_info(harp_plan_t plan, int64_t *d, int *m, int32_t *radix) {
     return HARP_OK;
 }
 
-int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group,
+int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group, int scale_mode,
                          const float *centroids) {
     if (!out) return HARP_ERR_INVALID_ARG;
     *out = nullptr;
     if (kind != HARP_LLOYD_MAX && kind != HARP_ABSMAX) return HARP_ERR_INVALID_ARG;
+    if (scale_mode != HARP_SCALE_RMS && scale_mode != HARP_SCALE_ABSMAX) return HARP_ERR_INVALID_ARG;
     if (bits < 2 || bits > 5) return HARP_ERR_UNSUPPORTED;
     if (group <= 0) return HARP_ERR_SHAPE;
     if (group % 32 != 0 || group > std::numeric_limits<int32_t>::max()) return HARP_ERR_UNSUPPORTED;
@@ -497,14 +502,20 @@ int harp_codebook_create(harp_codebook_t *out, int kind, int bits, int64_t group
             for (int k = 0; k < K; ++k) c[k] = centroids[k];
             for (int k = 0; k + 1 < K; ++k)
                 if (!(c[k] < c[k + 1])) { delete cb; return HARP_ERR_INVALID_ARG; }
+            if (scale_mode == HARP_SCALE_ABSMAX && !(c[K - 1] > 0.0f)) { delete cb; return HARP_ERR_INVALID_ARG; }
         } else {
             harp_lloyd_max_centroids(bits, c);
         }
         for (int k = 0; k < K; ++k) cb->q.level[k] = c[k];
         for (int k = 0; k + 1 < K; ++k)
             cb->q.thr[k] = static_cast<float>(0.5 * (static_cast<double>(c[k]) + static_cast<double>(c[k + 1])));
+        // default: RMS of the group; absmax mode: max |x| onto the largest centroid
+        cb->q.stat_max = (scale_mode == HARP_SCALE_ABSMAX) ? 1 : 0;
+        cb->q.scale_div = c[K - 1];
     } else {
         for (int k = 0; k < K; ++k) cb->q.level[k] = static_cast<float>(k - K / 2);
+        cb->q.stat_max = 1;
+        cb->q.scale_div = static_cast<float>((1 << (bits - 1)) - 1);
     }
     *out = cb;
     return HARP_OK;

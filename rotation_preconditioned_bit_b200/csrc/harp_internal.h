@@ -68,6 +68,8 @@ struct QuantDev {
     int kind;       // HARP_LLOYD_MAX | HARP_ABSMAX
     int bits;
     int group;
+    int stat_max;   // group statistic: 1 = max |x| (absmax, or Lloyd-Max with HARP_SCALE_ABSMAX), 0 = sum of squares
+    float scale_div;  // scale = statistic / scale_div when stat_max (qmax, or the largest centroid)
     float level[32];  // dequantised level per code (centroid or code - 2^(b-1))
     float thr[32];    // Lloyd-Max midpoints (K - 1 used)
 };

@@ -325,8 +325,9 @@ __device__ __forceinline__ void quantize_tile(const float *X, const Geo &g, cons
     constexpr int NWARP = NT / 32;
     const int d = g.d, gsz = Q.group, ng = d / gsz, nchunk = d >> 5, cpg = gsz >> 5;
     const int nrv = g.R / VW;
-    const bool is_max = (Q.kind == HARP_ABSMAX);
-    const bool lloyd = !is_max;
+    const bool is_max = Q.stat_max != 0;            // group statistic: max |x| or sum of squares
+    const bool lm = (Q.kind == HARP_LLOYD_MAX);
+    const bool lloyd = lm;
     // pass 1: statistics and scales, one (row group of VW rows, scale group) per warp
     for (int item = warp; item < nrv * ng; item += NWARP) {
         const int gi = item / nrv, rq = item - gi * nrv;
@@ -680,7 +681,8 @@ __device__ __forceinline__ void quantize_group(const QuantDev &Q, const void *in
                                                uint8_t *codes_row, uint16_t *scale, int64_t word0,
                                                int lane, const float (&t)[(1 << BITS) - 1]) {
     const int gsz = Q.group;
-    const bool is_max = (Q.kind == HARP_ABSMAX);
+    const bool is_max = Q.stat_max != 0;            // group statistic: max |x| or sum of squares
+    const bool lm = (Q.kind == HARP_LLOYD_MAX);
     float st = 0.0f;
     for (int c = 0; c < (gsz >> 5); ++c) st = combine(st, ldg1<PRO>(in, off + c * 32 + lane), is_max);
     st = warp_reduce(st, is_max);
@@ -690,7 +692,7 @@ __device__ __forceinline__ void quantize_group(const QuantDev &Q, const void *in
     const float is = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
     for (int c = 0; c < (gsz >> 5); ++c) {
         const float x = ldg1<PRO>(in, off + c * 32 + lane);
-        const int code = code_of<BITS>(x, s, is, !is_max, t);
+        const int code = code_of<BITS>(x, s, is, lm, t);
         const unsigned word = pack_words<BITS>(code, lane);
         if (lane < BITS) reinterpret_cast<unsigned *>(codes_row)[word0 + c * BITS + lane] = word;
     }

@@ -640,7 +640,8 @@ __device__ __forceinline__ void quantize_tile(const float *T, const PassDesc &D,
                                               const Tabs &tb, int warp, int lane) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     const int g = Q.group, ngt = Ec / g, per = g >> 5;
-    const bool is_max = (Q.kind == HARP_ABSMAX);
+    const bool is_max = Q.stat_max != 0;            // group statistic: max |x| or sum of squares
+    const bool lm = (Q.kind == HARP_LLOYD_MAX);
     float t[(1 << BITS) - 1];
 #pragma unroll
     for (int k = 0; k < (1 << BITS) - 1; ++k) t[k] = Q.thr[k];
@@ -664,7 +665,7 @@ __device__ __forceinline__ void quantize_tile(const float *T, const PassDesc &D,
         float *frow = F32COPY ? D.out_f32 + row * D.cols + c0 : nullptr;
         for (int e = 0; e < per; ++e) {
             const float x = rp[lane + 32 * e];
-            const int code = code_of<BITS>(x, s, inv, !is_max, t);
+            const int code = code_of<BITS>(x, s, inv, lm, t);
             const unsigned word = pack_words<BITS>(code, lane);
             if (lane < BITS) wrow[e * BITS + lane] = word;
             if constexpr (F32COPY) frow[32 * e + lane] = x;
@@ -757,7 +758,8 @@ __device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDes
                                                    int warp, int lane) {
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     const int g = Q.group, ngt = Ec / g, nit = g >> 5;
-    const bool is_max = (Q.kind == HARP_ABSMAX);
+    const bool is_max = Q.stat_max != 0;            // group statistic: max |x| or sum of squares
+    const bool lm = (Q.kind == HARP_LLOYD_MAX);
     const int64_t spr = D.cols / g;
     const int64_t wpr = D.cols * BITS / 32;
     const int q = lane >> 2, c = lane & 3;
@@ -796,7 +798,7 @@ __device__ __forceinline__ void quantize_tile_fast(const float *T, const PassDes
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     x[e] = rp[32 * it + e];
-                    word |= static_cast<unsigned>(code_of_smem<BITS>(x[e], s, inv, !is_max, ts)) << (BITS * e);
+                    word |= static_cast<unsigned>(code_of_smem<BITS>(x[e], s, inv, lm, ts)) << (BITS * e);
                 }
             }
             const int64_t col = c0 + 32 * it + 8 * c;       // first of this lane's 8 columns

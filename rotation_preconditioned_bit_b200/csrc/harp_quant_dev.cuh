@@ -23,14 +23,15 @@ __device__ __forceinline__ float warp_reduce(float v, bool is_max) {
     return v;
 }
 
-// Group scale from the combined statistic: RMS (Lloyd-Max) or absmax/qmax,
-// rounded to fp16 (nearest even), saturating at 65504.
+// Group scale from the combined statistic: RMS (sum of squares; Lloyd-Max's
+// default) or max|x| / scale_div (absmax: qmax; Lloyd-Max's absmax mode: the
+// largest centroid), rounded to fp16 (nearest even), saturating at 65504.
 __device__ __forceinline__ unsigned short group_scale_bits(float stat, const QuantDev &Q) {
     float s;
-    if (Q.kind == HARP_LLOYD_MAX) {
+    if (!Q.stat_max) {
         s = sqrtf(stat / static_cast<float>(Q.group));
     } else {
-        s = stat / static_cast<float>((1 << (Q.bits - 1)) - 1);
+        s = stat / Q.scale_div;
     }
     s = fminf(s, 65504.0f);
     return __half_as_ushort(__float2half_rn(s));

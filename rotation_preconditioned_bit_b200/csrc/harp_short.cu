@@ -202,7 +202,8 @@ __device__ __forceinline__ void quantize_rows(float *xr, const QuantDev &Q, cons
                                               const unsigned char *bins, bool use_bins, int d, int part,
                                               float *red, int v, bool mine, uint16_t *scales_row) {
     const int g = Q.group, ngr = d / g, nch = d / 32, lcpg = __ffs(g / 32) - 1;
-    const bool is_max = (Q.kind == HARP_ABSMAX);
+    const bool is_max = Q.stat_max != 0;            // group statistic: max |x| or sum of squares
+    const bool lm = (Q.kind == HARP_LLOYD_MAX);
     float st[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ci = 0; ci < MAXCH; ++ci) {
@@ -257,7 +258,7 @@ __device__ __forceinline__ void quantize_rows(float *xr, const QuantDev &Q, cons
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const unsigned code = static_cast<unsigned>(
-                        code_of_smem<BITS>(xr[ck * 32 + e], s, is, !is_max, thr));
+                        code_of_smem<BITS>(xr[ck * 32 + e], s, is, lm, thr));
                     const int bit = e * BITS, wi = bit >> 5, sh = bit & 31;
                     w[ci][wi] |= code << sh;
                     if (sh + BITS > 32) w[ci][wi + 1] |= code >> (32 - sh);

@@ -48,20 +48,20 @@ def test_plan_create_argument_checks():
     blk = np.zeros((16, 16, 16), np.float32)
     ptrs = (ctypes.POINTER(ctypes.c_float) * 2)(*(blk.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),) * 2)
     # product of radices != d
-    assert L.harp_plan_create(ctypes.byref(h), 255, 2, rad, ptrs, None) == 2
+    assert L.harp_plan_create(ctypes.byref(h), 255, 2, rad, ptrs, None, None) == 2
     # radix out of range
     rad_bad = (ctypes.c_int32 * 2)(65, 4)
-    assert L.harp_plan_create(ctypes.byref(h), 260, 2, rad_bad, ptrs, None) == 3
+    assert L.harp_plan_create(ctypes.byref(h), 260, 2, rad_bad, ptrs, None, None) == 3
     # too many stages
-    assert L.harp_plan_create(ctypes.byref(h), 256, 17, rad, ptrs, None) == 3
+    assert L.harp_plan_create(ctypes.byref(h), 256, 17, rad, ptrs, None, None) == 3
     # NULL pointers
-    assert L.harp_plan_create(None, 256, 2, rad, ptrs, None) == 1
-    assert L.harp_plan_create(ctypes.byref(h), 256, 2, None, ptrs, None) == 1
+    assert L.harp_plan_create(None, 256, 2, rad, ptrs, None, None) == 1
+    assert L.harp_plan_create(ctypes.byref(h), 256, 2, None, ptrs, None, None) == 1
     nullp = (ctypes.POINTER(ctypes.c_float) * 2)()
-    assert L.harp_plan_create(ctypes.byref(h), 256, 2, rad, nullp, None) == 1
+    assert L.harp_plan_create(ctypes.byref(h), 256, 2, rad, nullp, None, None) == 1
     # a vector too long for one CTA's shared memory
     rad_big = (ctypes.c_int32 * 2)(64, 1024)
-    assert L.harp_plan_create(ctypes.byref(h), 65536, 2, rad_big, ptrs, None) in (3, 2)
+    assert L.harp_plan_create(ctypes.byref(h), 65536, 2, rad_big, ptrs, None, None) in (3, 2)
 
 
 def test_plan_create_without_device_is_a_cuda_error(cuda_available):
@@ -72,7 +72,7 @@ def test_plan_create_without_device_is_a_cuda_error(cuda_available):
     rad = (ctypes.c_int32 * 2)(16, 16)
     blk = np.zeros((16, 16, 16), np.float32)
     ptrs = (ctypes.POINTER(ctypes.c_float) * 2)(*(blk.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),) * 2)
-    assert L.harp_plan_create(ctypes.byref(h), 256, 2, rad, ptrs, None) == 6
+    assert L.harp_plan_create(ctypes.byref(h), 256, 2, rad, ptrs, None, None) == 6
     assert not h.value
 
 

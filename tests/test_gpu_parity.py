@@ -502,3 +502,49 @@ def test_no_kernel_wait_ran_out():
     """Every wait inside the library's kernels is bounded and records when it
     runs out; none did during the tests above."""
     assert harp.harp_fault_status() == 0
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_lloyd_max_absmax_scale_mode_every_kernel(bits):
+    """The alternative Lloyd-Max scale s = max|x| / c_{K-1} (HARP_SCALE_ABSMAX)
+    in every quantizer the library has, against the oracle in the same mode:
+    the standalone codec, the two-sided pass kernels, the whole-vector kernel
+    (right-only rows of 4096) and the short-vector kernel (rows of 128)."""
+    group = 128
+    cb = harp.Codebook("lloyd_max", bits, group, scale_mode="absmax")
+    # standalone codec
+    X = synth.small_matrix(40 + bits, 33, 512, outlier_cols=3, scale=0.02).astype(np.float32)
+    oc, osc, m, sm = oracle.quantize("lloyd_max", bits, group, X.astype(np.float64), scale_mode="absmax")
+    codes, scales = harp.empty_codes(33, 512, cb)
+    harp.harp_quantize(cb, torch.from_numpy(X).cuda(), codes, scales)
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+    # two-sided pass kernels (1024 x 2048)
+    left_s = synth.side_draws(41, (16, 8, 8), "qr", synth.S_SIGNS_L, synth.S_BLOCKS_L)
+    right_s = synth.side_draws(41, (16, 16, 8), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    W = synth.small_matrix(42, 1024, 2048, outlier_cols=4, scale=0.02)
+    Wb = synth.to_bf16_bits(W)
+    Pl, Pr = oracle.processor(left_s), oracle.processor(right_s)
+    ref = Pr.rotate_rows(Pl.rotate_cols(synth.bf16_bits_to_f64(Wb)))
+    oc, osc, m, sm = oracle.quantize("lloyd_max", bits, group, ref, scale_mode="absmax")
+    left, right = harp.Plan.from_side(left_s), harp.Plan.from_side(right_s)
+    assert harp.harp_pass_count(left, right, cb) >= 2
+    xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, _ = harp.rotate_quantize(left, right, cb, xb)
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+    # whole-vector kernel: right-only rows of 4096
+    rs = synth.side_draws(43, (8, 8, 8, 8), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    Xr = synth.small_matrix(44, 40, 4096, outlier_cols=4).astype(np.float32)
+    P = oracle.processor(rs)
+    ref = P.rotate_rows(Xr.astype(np.float64))
+    oc, osc, m, sm = oracle.quantize("lloyd_max", bits, group, ref, scale_mode="absmax")
+    codes, scales, _ = harp.rotate_quantize(None, harp.Plan.from_side(rs), cb, torch.from_numpy(Xr).cuda())
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+    # short-vector kernel: rows of 128 (bf16 in)
+    h128 = harp.Plan((16, 8), [harp.stage_blocks("hadamard", b, 128 // b) for b in (16, 8)])
+    Ph = oracle.Processor((16, 8), [oracle.stage_blocks("hadamard", b, 128 // b) for b in (16, 8)])
+    Xs = synth.to_bf16_bits(synth.small_matrix(45, 600, 128, outlier_cols=2, scale=0.02))
+    ref = Ph.rotate_rows(synth.bf16_bits_to_f64(Xs))
+    oc, osc, m, sm = oracle.quantize("lloyd_max", bits, group, ref, scale_mode="absmax")
+    xs = torch.from_numpy(Xs.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, _ = harp.rotate_quantize(None, h128, cb, xs)
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
