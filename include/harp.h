@@ -355,7 +355,9 @@ int harp_set_block_stages(int mode);
  * second at most); a wait that runs out abandons the launch without trapping
  * and is recorded per device. This call returns that record for the current
  * device in *flags and clears it: 0 = no wait ran out; bit 0 = a tensor-core
- * batch of a two-sided call did not complete (that call's outputs are
+ * batch of a two-sided call did not complete; bit 1 = a bulk copy of a
+ * two-sided call's operand blocks or input did not arrive; bit 2 = a row
+ * tile of a right-only call did not arrive (those calls' outputs are
  * incomplete). Synchronous (it waits for the device's pending work).
  * Errors: INVALID_ARG (NULL flags), CUDA. */
 int harp_fault_status(unsigned int *flags);

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libharp.so")
 OBJDIR = os.path.join(HERE, "_build")
 SOURCES = [os.path.join(CSRC, f) for f in ("harp_kernels.cu", "harp_pass.cu", "harp_api.cpp", "harp_static_ws.cu",
-                                              "harp_theta.cu", "harp_short.cu")]
+                                              "harp_theta.cu", "harp_short.cu", "harp_rows.cu")]
 HEADERS = [os.path.join(CSRC, "harp_internal.h"), os.path.join(CSRC, "harp_quant_dev.cuh"),
            os.path.join(CSRC, "harp_tc.cuh"),
            os.path.join(INCLUDE, "harp.h")]

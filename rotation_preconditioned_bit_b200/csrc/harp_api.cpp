@@ -320,11 +320,15 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
     // host staging of the device layout
     const size_t sign_floats = (static_cast<size_t>(d) + 3) & ~static_cast<size_t>(3);
     size_t total = sign_floats;
-    std::vector<size_t> off(m), poff(m), uoff(m);
+    std::vector<size_t> off(m), poff(m), uoff(m), goff(m);
     for (int t = 0; t < m; ++t) {
         const int kpad = (radix[t] + 3) & ~3;
         off[t] = total;
         total += 2 * static_cast<size_t>(d) * kpad;   // fwd then inv
+    }
+    for (int t = 0; t < m; ++t) {                       // row-kernel layout
+        goff[t] = total;
+        total += static_cast<size_t>(d) * ((radix[t] + 3) & ~3);
     }
     for (int t = 0; t < m; ++t) {                       // pass-kernel layout
         const int b = radix[t];
@@ -351,6 +355,13 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
                     fwd[(c * b + j) * kpad + k] = B[k * b + j];
                     inv[(c * b + k) * kpad + j] = B[k * b + j];
                 }
+        }
+        float *gf = host.data() + goff[t];
+        for (int64_t c = 0; c < ng; ++c) {
+            const float *B = blocks[t] + c * b * b;
+            for (int k = 0; k < b; ++k)
+                for (int j = 0; j < b; ++j)
+                    gf[((static_cast<size_t>(j) * (kpad / 4) + k / 4) * ng + c) * 4 + (k & 3)] = B[k * b + j];
         }
         const int jp = pass_jpad(b), kp = pass_kp(b);
         float *pf = host.data() + poff[t];
@@ -414,6 +425,7 @@ int harp_plan_create(harp_plan_t *out, int64_t d, int m, const int32_t *radix,
         p->dev.st[t].s = s;
         p->dev.st[t].fwd = base + off[t];
         p->dev.st[t].inv = base + off[t] + static_cast<size_t>(d) * kpad;
+        p->dev.st[t].gfwd = base + goff[t];
         p->dev.st[t].jpad = pass_jpad(b);
         p->dev.st[t].kp = pass_kp(b);
         p->dev.st[t].pfwd = base + poff[t];
@@ -460,6 +472,7 @@ int harp_plan_load_theta(harp_plan_t plan, int stage, const int8_t *theta, float
     o.fwd = const_cast<float *>(sd.fwd);
     o.inv = const_cast<float *>(sd.inv);
     o.kpad = sd.kpad;
+    o.gfwd = const_cast<float *>(sd.gfwd);
     o.pfwd = const_cast<float *>(sd.pfwd);
     o.pinv = const_cast<float *>(sd.pinv);
     o.jp = sd.jpad;
@@ -658,6 +671,9 @@ int harp_rotate_quantize(harp_plan_t left, harp_plan_t right, harp_codebook_t cb
         S.scales = scales;
         return cuda_status(harp::launch_short(right->dev, cb->q, S, stream));
     }
+    if (!left && harp::rows_ok(right->dev, cb->q, in_dtype, in))
+        return cuda_status(harp::launch_rows(right->dev, cb->q, in, in_dtype, rows, codes, scales, rotated_out,
+                                             stream));
     if (use_passes(left, right, cb))
         return cuda_status(harp::launch_pass_fwd(left->dev, right->dev, cb->q, in, in_dtype, codes, scales,
                                                  rotated_out, static_cast<float *>(workspace), stream));
@@ -766,7 +782,11 @@ int harp_set_block_stages(int mode) {
 
 int harp_fault_status(unsigned int *flags) {
     if (!flags) return HARP_ERR_INVALID_ARG;
-    return cuda_status(harp::pass_fault_status(flags));
+    unsigned a = 0, b = 0;
+    int e = harp::pass_fault_status(&a);
+    if (e == 0) e = harp::rows_fault_status(&b);
+    *flags = a | b;
+    return cuda_status(e);
 }
 
 int harp_set_pass_events(void *const *events, int n) {

@@ -48,6 +48,12 @@ struct StageDev {
     int up;
     const float *ufwd;
     const float *uinv;
+    // The forward blocks interleaved across the stage's G = d/b groups for
+    // the row kernel, whose consecutive threads own consecutive groups:
+    //   gfwd[((j * kpad/4 + k/4) * G + c) * 4 + k%4] = B_{t,c}[k][j]
+    // (one float4 of four outputs' coefficients of input j per group, so a
+    // warp's 16-byte loads are contiguous), zero in the padding.
+    const float *gfwd;
 };
 
 // Operand float index of (row n, input kk) in a tensor-core block of
@@ -170,6 +176,7 @@ struct ThetaOut {
     float *ufwd;    // tensor-core operand blocks (StageDev::ufwd / uinv), up = padded size
     float *uinv;
     int up;
+    float *gfwd;    // group-interleaved forward blocks (StageDev::gfwd), same kpad
 };
 size_t theta_smem_bytes(int b);
 int launch_theta_blocks(int b, int64_t n_groups, const int8_t *theta, double scale,
@@ -197,6 +204,13 @@ struct ShortLaunch {
 };
 bool short_ok(const PlanDev &P, int mode, int in_bits);
 int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &L, void *stream);
+
+// Row kernel (harp_rows.cu): right-only rotate + quantize of whole rows for
+// processors with radices 2, 4, 8, 16 and d up to 8192 (contiguous rows).
+bool rows_ok(const PlanDev &P, const QuantDev &q, int in_dtype, const void *in);
+int launch_rows(const PlanDev &P, const QuantDev &q, const void *in, int in_dtype, int64_t rows, uint8_t *codes,
+                uint16_t *scales, float *rotated_out, void *stream);
+int rows_fault_status(unsigned *flags);
 
 // A plan's blocks live in device memory of the device that was current when
 // it was created; a launch from another device would read them through a

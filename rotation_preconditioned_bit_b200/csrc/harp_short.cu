@@ -170,8 +170,51 @@ __device__ __forceinline__ void stage_row(float *xr, const float *C, int b_rt, i
     }
 }
 
+// A stage whose blocks are all the normalised Sylvester Hadamard matrix H_b
+// (HARP section 2.2, theta = 0; PolarQuant section 2's H_128 is the product
+// of such stages): the fast Walsh-Hadamard butterfly, log2 b rounds of
+// (a + c, a - c) on inputs h apart, gives sum_j (-1)^popcount(k & j) x_j for
+// every output k; one multiply by the block entry 1/sqrt(b) follows. H_b is
+// symmetric, so the same code serves the inverse (B^T = B).
+template <int B>
+__device__ __forceinline__ void stage_row_fwht(float *xr, int s, int d, int part) {
+    const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(B)));
+    const int nh = d / (B * s);
+    int cidx = 0;
+    for (int h = 0; h < nh; ++h) {
+        for (int l = 0; l < s; ++l, ++cidx) {
+            if ((cidx & (NP - 1)) != part) continue;
+            float *base = xr + h * B * s + l;
+            float x[B];
+#pragma unroll
+            for (int j = 0; j < B; ++j) x[j] = base[j * s];
+#pragma unroll
+            for (int hh = 1; hh < B; hh <<= 1)
+#pragma unroll
+                for (int i = 0; i < B; ++i)
+                    if ((i & hh) == 0) {
+                        const float a = x[i], c = x[i + hh];
+                        x[i] = a + c;
+                        x[i + hh] = a - c;
+                    }
+#pragma unroll
+            for (int j = 0; j < B; ++j) base[j * s] = x[j] * scale;
+        }
+    }
+}
+
 __device__ __forceinline__ void run_stage_row(float *xr, const float *C, const StageDev &S, int d, int part) {
     const int b = S.b, kp = S.kpad, s = static_cast<int>(S.s);
+    if (S.had) {
+        switch (b) {
+            case 2: stage_row_fwht<2>(xr, s, d, part); return;
+            case 4: stage_row_fwht<4>(xr, s, d, part); return;
+            case 8: stage_row_fwht<8>(xr, s, d, part); return;
+            case 16: stage_row_fwht<16>(xr, s, d, part); return;
+            case 32: stage_row_fwht<32>(xr, s, d, part); return;
+            default: break;
+        }
+    }
     switch (b) {
         case 4: stage_row<4, true>(xr, C, b, kp, s, d, part); break;
         case 8: stage_row<8, true>(xr, C, b, kp, s, d, part); break;

@@ -98,6 +98,7 @@ theta_blocks_kernel(int b, int64_t n_groups, const int8_t *__restrict__ theta, d
             if (o.plain) o.plain[(c * b + k) * b + j] = v;
             if (o.fwd) o.fwd[(c * b + j) * o.kpad + k] = v;
             if (o.inv) o.inv[(c * b + k) * o.kpad + j] = v;
+            if (o.gfwd) o.gfwd[((j * (o.kpad >> 2) + (k >> 2)) * n_groups + c) * 4 + (k & 3)] = v;
             if (o.pfwd) o.pfwd[(c * o.jp + j) * o.kp + k] = v;
             if (o.pinv) o.pinv[(c * o.jp + k) * o.kp + j] = v;
             if (o.ufwd || o.uinv) {

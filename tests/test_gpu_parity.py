@@ -169,6 +169,34 @@ def test_c3_activation_rows(T):
     assert rel_l2(xb.float().cpu().numpy(), ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("radix,rows,dtype", [((16, 16, 16), 37, "f32"), ((4, 8, 16, 2, 8), 61, "bf16"),
+                                              ((2, 4, 8, 16), 1000, "bf16"), ((16, 16), 9, "f32")])
+@pytest.mark.parametrize("kind,bits,group", [("lloyd_max", 3, 128), ("absmax", 4, 256), ("lloyd_max", 2, 64)])
+def test_row_kernel_shapes(radix, rows, dtype, kind, bits, group):
+    """Right-only rotate + quantize of whole rows (the row kernel: radices 2, 4,
+    8, 16) on ragged row counts, fp32 and bf16 inputs, several group sizes,
+    with the fp32 rotated copy, against the oracle element by element."""
+    d = int(np.prod(radix))
+    if d % group:
+        pytest.skip("group does not divide the row")
+    s = synth.side_draws(90 + d, radix, "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    X = synth.small_matrix(91 + rows, rows, d, outlier_cols=3, scale=0.02)
+    if dtype == "bf16":
+        Xb = synth.to_bf16_bits(X)
+        x = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).cuda()
+        Xf = synth.bf16_bits_to_f64(Xb)
+    else:
+        X32 = X.astype(np.float32)
+        x = torch.from_numpy(X32).cuda()
+        Xf = X32.astype(np.float64)
+    P = oracle.processor(s)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(Xf, None, P, kind, bits, group)
+    cb = harp.Codebook(kind, bits, group)
+    codes, scales, rot = harp.rotate_quantize(None, harp.Plan.from_side(s), cb, x, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+
+
 # ------------------------------------------------------------ inverse paths, whole matrices
 
 def _inverse_full(w, left, right, q, raw, sc, Pl, Pr, label):
@@ -531,14 +559,16 @@ def test_lloyd_max_absmax_scale_mode_every_kernel(bits):
     xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
     codes, scales, _ = harp.rotate_quantize(left, right, cb, xb)
     compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
-    # whole-vector kernel: right-only rows of 4096
-    rs = synth.side_draws(43, (8, 8, 8, 8), "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
-    Xr = synth.small_matrix(44, 40, 4096, outlier_cols=4).astype(np.float32)
-    P = oracle.processor(rs)
-    ref = P.rotate_rows(Xr.astype(np.float64))
-    oc, osc, m, sm = oracle.quantize("lloyd_max", bits, group, ref, scale_mode="absmax")
-    codes, scales, _ = harp.rotate_quantize(None, harp.Plan.from_side(rs), cb, torch.from_numpy(Xr).cuda())
-    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
+    # right-only rows: the row kernel (radices 8) and the whole-vector kernel (a radix 7)
+    for radix in ((8, 8, 8, 8), (8, 8, 8, 7)):
+        rs = synth.side_draws(43, radix, "qr", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+        d = int(np.prod(radix))
+        Xr = synth.small_matrix(44, 40, d, outlier_cols=4).astype(np.float32)
+        P = oracle.processor(rs)
+        ref = P.rotate_rows(Xr.astype(np.float64))
+        oc, osc, m, sm = oracle.quantize("lloyd_max", bits, group, ref, scale_mode="absmax")
+        codes, scales, _ = harp.rotate_quantize(None, harp.Plan.from_side(rs), cb, torch.from_numpy(Xr).cuda())
+        compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, bits, group)
     # short-vector kernel: rows of 128 (bf16 in)
     h128 = harp.Plan((16, 8), [harp.stage_blocks("hadamard", b, 128 // b) for b in (16, 8)])
     Ph = oracle.Processor((16, 8), [oracle.stage_blocks("hadamard", b, 128 // b) for b in (16, 8)])

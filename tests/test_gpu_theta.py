@@ -136,6 +136,31 @@ def test_loaded_plans_rotate_and_quantize_like_the_oracle():
                   Pl.rotate_cols(X.astype(np.float32).astype(np.float64), inverse=True)) <= TOL_F32
 
 
+def test_loaded_plan_feeds_the_row_kernel():
+    """A right-only rotate + quantize whose radices (16, 8, 4) take the row
+    kernel, which reads the plan's group-interleaved copy of the forward
+    blocks: after every stage is replaced from int8 parameters, the rotated
+    rows, codes and scales match the oracle's processor built from the same
+    parameters."""
+    torch.cuda.set_device(0)
+    radix = (16, 8, 4)
+    rows, cols = 300, 512
+    side = synth.side_draws(81, radix, "hadamard", synth.S_SIGNS_R, synth.S_BLOCKS_R)
+    plan = harp.Plan.from_side(side)
+    params = _theta_side(82, radix, 20)
+    _load(plan, params)
+    P = _oracle_processor(radix, params, side.signs)
+    W = synth.small_matrix(83, rows, cols, outlier_cols=3, scale=0.02)
+    Wb = synth.to_bf16_bits(W)
+    X = synth.bf16_bits_to_f64(Wb)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(X, None, P, "absmax", 4, 128)
+    cb = harp.Codebook("absmax", 4, 128)
+    xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, rot = harp.rotate_quantize(None, plan, cb, xb, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16), oc, osc, m, sm, 4, 128)
+
+
 def test_load_is_stream_ordered_and_rejects_bad_stage():
     """A rotation launched before a load on the same stream sees the old
     blocks, one launched after it the new ones; a stage outside [0, m) is an
