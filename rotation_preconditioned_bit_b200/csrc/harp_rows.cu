@@ -71,10 +71,12 @@ struct RowsDesc {
     int stage_base, part_base, bar_base, lev_base;   // float offsets in shared memory
 };
 
-// The tile stores coordinate a of a row at a + a/8 (one pad word per 8): a
-// stage whose groups are 8 or 64 coordinates apart then spreads a warp's 32
-// lanes over 32 banks, and 8 consecutive coordinates stay contiguous.
-__host__ __device__ __forceinline__ int sk(int a) { return a + (a >> 3); }
+// The tile stores coordinate a of a row at a XOR-swizzled word of the same
+// 32-word block: a ^ ((a/32) % 8 + 8 * ((a/64) % 4)). A warp then reads 32
+// consecutive coordinates, 32 coordinates 8 apart, or 4 runs of 8 that are
+// 64 apart (the groups of the stages of a radix-8 processor, and the
+// quantizer's lanes) from 32 different banks.
+__host__ __device__ __forceinline__ int sk(int a) { return a ^ (((a >> 5) & 7) | (((a >> 6) & 3) << 3)); }
 
 typedef unsigned long long f2_t;
 
@@ -165,26 +167,25 @@ __device__ __forceinline__ void stage_rows(float *T, const RowsDesc &D, int t, i
 template <int B, int RT>
 __device__ __forceinline__ void stage_rows_rc(float *T, const RowsDesc &D, int t, int nrows, int tid) {
     static_assert(B == 2 || B == 4 || B == 8, "register-resident blocks take radices 2, 4 and 8");
-    const int s = D.s[t], sl = D.sl[t], kp = D.kpad[t];
+    const int s = D.s[t], sl = D.sl[t], kq = D.kpad[t] >> 2;
     const int G = D.d / B;
     const int GT = G < RT_THREADS ? G : RT_THREADS;
     const int RS = RT_THREADS / GT;
     const int rs = tid / GT;
     if (rs >= RS) return;
-    const float *coef = D.gfwd[t];
     const int pitch = D.pitch;
     for (int g = tid - rs * GT; g < G; g += GT) {
         const int h = g >> sl, l = g & (s - 1);
         const int base = h * B * s + l;
         // group g's float4 for (input j, outputs 4q..4q+3) sits at
-        // ((j * kp/4 + q) * G + g): consecutive threads, consecutive float4s
-        const float4 *cp = reinterpret_cast<const float4 *>(coef) + g;
+        // ((j * kpad/4 + q) * G + g): consecutive threads, consecutive float4s
+        const float4 *cp = reinterpret_cast<const float4 *>(D.gfwd[t]) + g;
         f2_t cc[B][B / 2];
 #pragma unroll
         for (int j = 0; j < B; ++j) {
 #pragma unroll
             for (int q = 0; q < (B + 3) / 4; ++q) {
-                const float4 v = __ldg(cp + static_cast<int64_t>(j * (kp >> 2) + q) * G);
+                const float4 v = __ldg(cp + static_cast<int64_t>(j * kq + q) * G);
                 cc[j][2 * q] = f2_pack(v.x, v.y);
                 if constexpr (B >= 4) cc[j][2 * q + 1] = f2_pack(v.z, v.w);
             }
@@ -276,26 +277,43 @@ __device__ __forceinline__ void stage_rows_any(float *T, const RowsDesc &D, int 
     }
 }
 
-// Staged input rows -> fp32 tile, times the sign vector.
+// Staged input rows -> fp32 tile, times the sign vector: each thread takes
+// columns c..c+3 (c a multiple of 4) of every row, its signs loaded once.
 __device__ __forceinline__ void convert_rows(const RowsDesc &D, const void *S, float *T, int nrows, int tid) {
-    const int d = D.d, nq = nrows * (d >> 2);
-    for (int i = tid; i < nq; i += RT_THREADS) {
-        const int r = i / (d >> 2), c = 4 * (i - r * (d >> 2));
-        float4 x;
-        if (D.in_bf16) {
-            const uint2 u = *reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(S) + r * d + c);
-            x = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                            __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-        } else {
-            x = *reinterpret_cast<const float4 *>(static_cast<const float *>(S) + r * d + c);
-        }
+    const int d = D.d;
+    for (int c = 4 * tid; c < d; c += 4 * RT_THREADS) {
         const float4 sg = __ldg(reinterpret_cast<const float4 *>(D.signs + c));
-        float *t = T + r * D.pitch + sk(c);      // c..c+3 stay contiguous (c is a multiple of 4)
-        t[0] = x.x * sg.x;
-        t[1] = x.y * sg.y;
-        t[2] = x.z * sg.z;
-        t[3] = x.w * sg.w;
+        const int p0 = sk(c), p1 = sk(c + 1), p2 = sk(c + 2), p3 = sk(c + 3);
+#pragma unroll 4
+        for (int r = 0; r < nrows; ++r) {
+            float4 x;
+            if (D.in_bf16) {
+                const uint2 u = *reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(S) + r * d + c);
+                x = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+            } else {
+                x = *reinterpret_cast<const float4 *>(static_cast<const float *>(S) + r * d + c);
+            }
+            float *t = T + r * D.pitch;
+            t[p0] = x.x * sg.x;
+            t[p1] = x.y * sg.y;
+            t[p2] = x.z * sg.z;
+            t[p3] = x.w * sg.w;
+        }
     }
+}
+
+// Absmax code of z = x / scale: clamp to [-qmax, qmax], then the nearest
+// integer with ties to even (adding 1.5 * 2^23 leaves it in the low mantissa
+// bits; exact for |z| < 2^22, and the clamp keeps |z| <= qmax), plus 2^(b-1).
+// The same code as rint(z) clamped; a zero scale gives inv = 0, z = 0 and
+// the mid code.
+template <int BITS>
+__device__ __forceinline__ int absmax_code(float x, float inv) {
+    constexpr int HALF = 1 << (BITS - 1);
+    constexpr float QMAX = static_cast<float>(HALF - 1);
+    const float z = fminf(fmaxf(x * inv, -QMAX), QMAX);
+    return (__float_as_int(z + 12582912.0f) - 0x4B400000) + HALF;
 }
 
 // Quantise the tile's rows: chunks of D.chunk coordinates (whole chunks per
@@ -345,15 +363,21 @@ __device__ __forceinline__ void quantize_rows(const float *T, const RowsDesc &D,
             // so lanes past the chunk's end simply skip the loop
             constexpr int PER = 32 / BITS;
             for (int col = c * ch + PER * lane; col < (c + 1) * ch; col += 32 * PER) {
-                const float *xp = x + sk(col);
-                unsigned word = 0;
                 float v[PER];
 #pragma unroll
-                for (int i = 0; i < PER; ++i) {
-                    v[i] = xp[i + (i >> 3)];      // col is a multiple of 8: one pad word per 8
-                    const int code = binned ? code_binned<64>(v[i] * inv, ts, bins)
-                                            : code_of_smem<BITS>(v[i], sc, inv, lm, ts);
-                    word |= static_cast<unsigned>(code) << (BITS * i);
+                for (int i = 0; i < PER; ++i) v[i] = x[sk(col + i)];
+                unsigned word = 0;
+                if (!lm) {
+#pragma unroll
+                    for (int i = 0; i < PER; ++i) word |= static_cast<unsigned>(absmax_code<BITS>(v[i], inv)) << (BITS * i);
+                } else if (binned) {
+#pragma unroll
+                    for (int i = 0; i < PER; ++i)
+                        word |= static_cast<unsigned>(code_binned<64>(v[i] * inv, ts, bins)) << (BITS * i);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < PER; ++i)
+                        word |= static_cast<unsigned>(code_of_smem<BITS>(v[i], sc, inv, true, ts)) << (BITS * i);
                 }
                 wrow[col / PER] = word;
                 if (frow) {
@@ -366,7 +390,8 @@ __device__ __forceinline__ void quantize_rows(const float *T, const RowsDesc &D,
             for (int e = 0; e < cw; ++e) {
                 const int col = c * ch + 32 * e + lane;
                 const float v = x[sk(col)];
-                const int code = binned ? code_binned<64>(v * inv, ts, bins) : code_of_smem<BITS>(v, sc, inv, lm, ts);
+                const int code = !lm ? absmax_code<BITS>(v, inv)
+                                 : binned ? code_binned<64>(v * inv, ts, bins) : code_of_smem<BITS>(v, sc, inv, true, ts);
                 const unsigned word = pack_words<BITS>(code, lane);
                 if (lane < BITS) wrow[static_cast<int64_t>(c) * cw * BITS + e * BITS + lane] = word;
                 if (frow) frow[col] = v;
@@ -466,7 +491,7 @@ RowsGeom rows_geom(const PlanDev &P, int in_dtype, const QuantDev &q) {
     int bmax = 1;
     for (int t = 0; t < P.m; ++t) bmax = std::max(bmax, P.st[t].b);
     const int esize = in_dtype == HARP_BF16 ? 2 : 4;
-    g.pitch = ((sk(d) + 3) & ~3) + 4;
+    g.pitch = d + 4;
     g.chunk = std::min(q.group, 1024);
     while (q.group % g.chunk) g.chunk >>= 1;
     for (int R = std::min(8, 64 / bmax); R >= 1; R >>= 1) {
