@@ -57,7 +57,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # L2 when a launch ends are counted by the next launch. When the pass-kernel
 # source differs from the captured one the figures no longer describe the
 # kernel and the roofline's traffic field is reported as null.
-MEASURED_TRAFFIC = {"kernel_src": None, "bytes": {}}
+MEASURED_TRAFFIC = {"kernel_src": "025b4495f0849231", "bytes": {
+    "fwd_p0_2bit": 49889024,
+    "fwd_p1_2bit": 86765824,
+    "fwd_p2_2bit": 68017152,
+    "inv_p0_2bit": 16860672,
+    "inv_p1_2bit": 86633984,
+    "inv_p2_2bit": 69223424,
+    "fwd_p0_4bit": 47279616,
+    "fwd_p1_4bit": 86482688,
+    "fwd_p2_4bit": 68010496,
+    "inv_p0_4bit": 21036032,
+    "inv_p1_4bit": 86616576,
+    "inv_p2_4bit": 69220096,
+}}
 PASS_SRC = os.path.join(ROOT, "rotation_preconditioned_bit_b200", "csrc", "harp_pass.cu")
 
 
@@ -365,10 +378,12 @@ def run_gpu(args, rank, world, local_rank):
 WORKLOAD_NAMES = ("c1", "c3", "c4", "c5", "rht", "pq", "theta")
 
 
-def run_workloads(steps, dev, names=WORKLOAD_NAMES):
+def run_workloads(steps, dev, names=WORKLOAD_NAMES, c3_tokens=(1, 16, 256, 8192)):
     """The other synthetic workloads, through the public calls with inputs
     resident on the device: per call, mean device time over `steps` calls
-    (CUDA events; L2 not flushed: each call streams more than L2 except c1),
+    (CUDA events; L2 not flushed: each call streams more than L2 except c1
+    and the small token counts, which also report fwd_graph_us, the time per
+    call replayed from a CUDA graph),
     algorithmic GB/s (input read + codes + scales written for a forward;
     codes + scales read + output written for an inverse) and elements/s."""
     import numpy as np
@@ -389,12 +404,38 @@ def run_workloads(steps, dev, names=WORKLOAD_NAMES):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / steps * 1e-3
 
+    def graph_timed(fn, calls=20, reps=5):
+        """Device time per call with the calls replayed from a CUDA graph
+        (no host work between launches): the latency a serving loop that
+        captures its steps sees; for small calls the plain loop above is
+        bound by the host's per-call overhead instead."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(calls):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / (reps * calls) * 1e-3
+
     out = {}
     jobs = []
     for name in [n for n in ("c1", "c3", "c4", "c5", "rht") if n in names]:
         # the activation workload at every token count (T <= 16 is a
         # latency case: its time in microseconds is the figure to read)
-        jobs += [(name, T) for T in (1, 16, 256, 8192)] if name == "c3" else [(name, None)]
+        jobs += [(name, T) for T in c3_tokens] if name == "c3" else [(name, None)]
     for name, tokens in jobs:
         if name == "rht":
             # the c2 weight with Hadamard-initialised processors on both sides
@@ -427,6 +468,9 @@ def run_workloads(steps, dev, names=WORKLOAD_NAMES):
             t = timed(lambda: harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws))
             rec = {"shape": [rows, cols], "fwd_us": round(t * 1e6, 2),
                    "fwd_gbs": round(n * (in_b + code_b) / t / 1e9, 2), "fwd_elems_per_s": float(f"{n / t:.4g}")}
+            if rows * cols <= 256 * 4096:
+                tg = graph_timed(lambda: harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws))
+                rec["fwd_graph_us"] = round(tg * 1e6, 2)
             if left is not None:
                 o = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
                 t = timed(lambda: harp.harp_dequantize_unrotate(left, right, cb, codes, scales, o, ws))
@@ -641,6 +685,8 @@ def main():
     ap.add_argument("--workloads-only", default=None, metavar="NAMES",
                     help="time only these workloads (comma list of " + ",".join(WORKLOAD_NAMES) +
                          ") on one GPU, print them as one JSON line and exit")
+    ap.add_argument("--c3-tokens", default="1,16,256,8192", metavar="LIST",
+                    help="token counts of the c3 activation workload (comma list)")
     args = ap.parse_args()
     if args.workloads_only is not None:
         import torch
@@ -649,7 +695,8 @@ def main():
         if bad:
             ap.error(f"unknown workloads {bad}")
         torch.cuda.set_device(0)
-        print(json.dumps({"workloads": run_workloads(max(3, args.steps), torch.device("cuda", 0), names)}))
+        toks = tuple(int(v) for v in args.c3_tokens.split(",") if v)
+        print(json.dumps({"workloads": run_workloads(max(3, args.steps), torch.device("cuda", 0), names, toks)}))
         return
     args.warmup = max(3, args.warmup)
 

@@ -483,9 +483,9 @@ struct RowsGeom {
 };
 
 // Tile rows and shared-memory layout for d coordinates, or R = 0 when the
-// rows do not fit. R is a power of two, at most 64 / (largest radix) so a
-// thread's accumulators fit its registers.
-RowsGeom rows_geom(const PlanDev &P, int in_dtype, const QuantDev &q) {
+// rows do not fit. R is a power of two, at most rmax and 64 / (largest
+// radix) so a thread's accumulators fit its registers.
+RowsGeom rows_geom(const PlanDev &P, int in_dtype, const QuantDev &q, int rmax = 8) {
     RowsGeom g{};
     const int d = static_cast<int>(P.d);
     int bmax = 1;
@@ -494,7 +494,7 @@ RowsGeom rows_geom(const PlanDev &P, int in_dtype, const QuantDev &q) {
     g.pitch = d + 4;
     g.chunk = std::min(q.group, 1024);
     while (q.group % g.chunk) g.chunk >>= 1;
-    for (int R = std::min(8, 64 / bmax); R >= 1; R >>= 1) {
+    for (int R = std::min(rmax, 64 / bmax); R >= 1; R >>= 1) {
         g.R = R;
         g.stage_base = ((R * g.pitch) + 31) & ~31;
         g.part_base = g.stage_base + ((R * d * esize / 4 + 31) & ~31);
@@ -523,7 +523,25 @@ bool rows_ok(const PlanDev &P, const QuantDev &q, int in_dtype, const void *in) 
 
 int launch_rows(const PlanDev &P, const QuantDev &q, const void *in, int in_dtype, int64_t rows, uint8_t *codes,
                 uint16_t *scales, float *rotated_out, void *stream) {
-    const RowsGeom g = rows_geom(P, in_dtype, q);
+    static int attr_done[64] = {};
+    static int nsm[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        e = cudaFuncSetAttribute(rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROWS_SMEM_BUDGET);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&nsm[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = 1;
+    }
+    if (rows == 0) return cudaSuccess;
+    // tiles as small as keep every SM busy: a tile's rows go through the
+    // stages one after another, so a few rows finish sooner on more SMs
+    int rmax = 1;
+    while (rmax < 8 && static_cast<int64_t>(rmax) * nsm[dev] < rows) rmax <<= 1;
+    const RowsGeom g = rows_geom(P, in_dtype, q, rmax);
     if (g.R == 0) return cudaErrorInvalidValue;
     RowsDesc D{};
     D.d = static_cast<int>(P.d);
@@ -552,20 +570,6 @@ int launch_rows(const PlanDev &P, const QuantDev &q, const void *in, int in_dtyp
     D.part_base = g.part_base;
     D.lev_base = g.lev_base;
     D.bar_base = g.bar_base;
-    static int attr_done[64] = {};
-    static int nsm[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
-        e = cudaFuncSetAttribute(rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROWS_SMEM_BUDGET);
-        if (e != cudaSuccess) return e;
-        e = cudaDeviceGetAttribute(&nsm[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = 1;
-    }
-    if (rows == 0) return cudaSuccess;
     const int64_t ntiles = (rows + g.R - 1) / g.R;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, nsm[dev]));
     rows_kernel<<<grid, RT_THREADS, g.smem, static_cast<cudaStream_t>(stream)>>>(D, q, bins_exact(q, 64) ? 1 : 0);
