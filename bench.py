@@ -378,7 +378,57 @@ def run_gpu(args, rank, world, local_rank):
 WORKLOAD_NAMES = ("c1", "c3", "c4", "c5", "rht", "pq", "theta")
 
 
-def run_workloads(steps, dev, names=WORKLOAD_NAMES, c3_tokens=(1, 16, 256, 8192)):
+def workload_cpu_baseline(w, q, budget_s=1.0):
+    """The float64 oracle on a bounded sample of a workload's forward call,
+    on all host cores (OpenMP over rows / columns) and on one thread: the
+    right pass + quantise + pack on a strip of rows and, for two-sided
+    calls, the left pass on a strip of columns, each the same fraction of the
+    matrix (sized to about budget_s seconds). Credited with that fraction of
+    the call's algorithmic bytes."""
+    import numpy as np
+
+    import oracle
+    from rotation_preconditioned_bit_b200 import synth
+
+    rows, cols = w.rows, w.cols
+    Pr = oracle.processor(w.right)
+    Pl = oracle.processor(w.left) if w.left is not None else None
+    in_b = 2 if w.dtype == "bf16" else 4
+
+    def f64(a):
+        return synth.bf16_bits_to_f64(a) if w.dtype == "bf16" else np.asarray(a, dtype=np.float64)
+
+    def sample(frac):
+        nr = max(1, int(round(rows * frac)))
+        nc = max(1, int(round(cols * frac)))
+        Xr = f64(np.ascontiguousarray(w.x[:nr]))
+        Xc = f64(np.ascontiguousarray(w.x[:, :nc])) if Pl is not None else None
+        t0 = time.perf_counter()
+        if Pl is not None:
+            Pl.rotate_cols(Xc)
+        Y = Pr.rotate_rows(Xr)
+        codes, scales, _, _ = oracle.quantize(q.kind, q.bits, q.group, Y, with_margins=False)
+        oracle.pack(q.bits, codes)
+        dt = time.perf_counter() - t0
+        return dt, nr * cols, nr, nc
+
+    out = {}
+    cores = os.cpu_count() or 1
+    for label, nt in (("all_cores", cores), ("single_thread", 1)):
+        oracle.threads(nt)
+        frac = min(1.0, (1 << 18) / (rows * cols))
+        dt, _, _, _ = sample(frac)
+        frac = min(1.0, frac * budget_s / max(dt, 1e-3))
+        dt, elems, nr, nc = sample(frac)
+        gbs = elems * (in_b + q.bits / 8.0 + 2.0 / q.group) / dt / 1e9
+        strip = f"{nr}x{cols} row strip" + (f" and {rows}x{nc} column strip" if Pl is not None else "")
+        out[label] = {"gbs": round(gbs, 4), "cores": oracle.threads(), "seconds": round(dt, 2),
+                      "sample": f"float64 oracle, forward on a {strip} ({frac:.4f} of the matrix)"}
+    oracle.threads(cores)
+    return out
+
+
+def run_workloads(steps, dev, names=WORKLOAD_NAMES, c3_tokens=(1, 16, 256, 8192), cpu=False):
     """The other synthetic workloads, through the public calls with inputs
     resident on the device: per call, mean device time over `steps` calls
     (CUDA events; L2 not flushed: each call streams more than L2 except c1
@@ -471,6 +521,8 @@ def run_workloads(steps, dev, names=WORKLOAD_NAMES, c3_tokens=(1, 16, 256, 8192)
             if rows * cols <= 256 * 4096:
                 tg = graph_timed(lambda: harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws))
                 rec["fwd_graph_us"] = round(tg * 1e6, 2)
+            if cpu:
+                rec["cpu_oracle"] = workload_cpu_baseline(w, q)
             if left is not None:
                 o = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
                 t = timed(lambda: harp.harp_dequantize_unrotate(left, right, cb, codes, scales, o, ws))
@@ -687,6 +739,9 @@ def main():
                          ") on one GPU, print them as one JSON line and exit")
     ap.add_argument("--c3-tokens", default="1,16,256,8192", metavar="LIST",
                     help="token counts of the c3 activation workload (comma list)")
+    ap.add_argument("--workload-cpu", action="store_true",
+                    help="with --workloads-only: also time the float64 oracle on a bounded sample of each "
+                         "forward call (all host cores and one thread, about 1 s each)")
     args = ap.parse_args()
     if args.workloads_only is not None:
         import torch
@@ -696,7 +751,8 @@ def main():
             ap.error(f"unknown workloads {bad}")
         torch.cuda.set_device(0)
         toks = tuple(int(v) for v in args.c3_tokens.split(",") if v)
-        print(json.dumps({"workloads": run_workloads(max(3, args.steps), torch.device("cuda", 0), names, toks)}))
+        print(json.dumps({"workloads": run_workloads(max(3, args.steps), torch.device("cuda", 0), names, toks,
+                                                     cpu=args.workload_cpu)}))
         return
     args.warmup = max(3, args.warmup)
 
