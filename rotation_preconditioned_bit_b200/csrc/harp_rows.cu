@@ -332,8 +332,19 @@ __device__ __forceinline__ void quantize_rows(const float *T, const RowsDesc &D,
     for (int it = warp; it < items; it += RT_WARPS) {
         const int r = it / nch, c = it - r * nch;
         const float *x = T + r * D.pitch;
-        float st = 0.0f;
-        for (int e = 0; e < cw; ++e) st = combine(st, x[sk(c * ch + 32 * e + lane)], is_max);
+        // a chunk is whole 32-word swizzle blocks, so its words hold exactly
+        // its values (in another order): the statistic reads them linearly,
+        // four per 16-byte load, combined in a fixed order
+        const float4 *xv = reinterpret_cast<const float4 *>(x + c * ch);
+        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+        for (int e = lane; e < ch / 4; e += 32) {
+            const float4 v = xv[e];
+            a0 = combine(a0, v.x, is_max);
+            a1 = combine(a1, v.y, is_max);
+            a2 = combine(a2, v.z, is_max);
+            a3 = combine(a3, v.w, is_max);
+        }
+        float st = is_max ? fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) : (a0 + a1) + (a2 + a3);
         st = warp_reduce(st, is_max);
         if (lane == 0) part[it] = st;
     }
@@ -362,10 +373,15 @@ __device__ __forceinline__ void quantize_rows(const float *T, const RowsDesc &D,
             // PER consecutive codes fill one 32-bit word; no cross-lane step,
             // so lanes past the chunk's end simply skip the loop
             constexpr int PER = 32 / BITS;
+#pragma unroll 4
             for (int col = c * ch + PER * lane; col < (c + 1) * ch; col += 32 * PER) {
+                // col .. col + PER - 1 share one 32-word block and so one
+                // swizzle mask m: coordinate col + i sits at (col ^ m) ^ i
+                const int blk = col >> 5;
+                const int sw = col ^ ((blk & 7) | (((blk >> 1) & 3) << 3));
                 float v[PER];
 #pragma unroll
-                for (int i = 0; i < PER; ++i) v[i] = x[sk(col + i)];
+                for (int i = 0; i < PER; ++i) v[i] = x[sw ^ i];
                 unsigned word = 0;
                 if (!lm) {
 #pragma unroll
