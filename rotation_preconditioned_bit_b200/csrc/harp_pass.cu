@@ -130,6 +130,7 @@ struct PassDesc {
     FDiv f_gch;         // ... by the 32-code chunks of a quantiser group
     FDiv f_nq;          // ... by the column quads of a tile row
     FDiv f_nchc;        // ... by the 32-column chunks of a tile row (codes)
+    FDiv f_nchc4;       // ... by the groups of 4 such chunks
     int stage_base;     // float offset of the staging buffer of the next tile's input
     int coef_base;      // float offset of the coefficient area
     int coef_floats;
@@ -1033,6 +1034,25 @@ __device__ __forceinline__ void decode_staged(const PassDesc &D, const QuantDev 
     const int Er = D.ax[0].E, Ec = D.ax[1].E, TCp = D.TCp;
     const int nch = Ec >> 5, wpr = nch * BITS, ngt = Ec / Q.group;
     const int bit = lane * BITS, wi = bit >> 5, sh = bit & 31;
+    if ((nch & 3) == 0) {
+        // a warp unit is one row's 4 consecutive 32-column chunks: each lane
+        // decodes column `lane` of each (consecutive lanes store consecutive
+        // columns), with the row's index arithmetic paid once per 4 codes
+        const int nu4 = nch >> 2;
+        for (int u = warp; u < Er * nu4; u += PW) {
+            const int tr = static_cast<int>(fdiv(static_cast<unsigned>(u), D.f_nchc4)), ch0 = 4 * (u - tr * nu4);
+            const uint32_t *wsrc = S + tr * wpr + ch0 * BITS;
+            const float *srow = ssc + tr * ngt;
+            float *trow = T + tr * TCp + ch0 * 32 + lane;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                unsigned code = wsrc[k * BITS + wi] >> sh;
+                if (sh + BITS > 32) code |= wsrc[k * BITS + wi + 1] << (32 - sh);
+                trow[32 * k] = srow[fdiv(static_cast<unsigned>(ch0 + k), D.f_gch)] * lev[code & MASK];
+            }
+        }
+        return;
+    }
     for (int u = warp; u < Er * nch; u += PW) {
         const int tr = static_cast<int>(fdiv(static_cast<unsigned>(u), D.f_nchc)), ch = u - tr * nch;
         const uint32_t *wsrc = S + tr * wpr + ch * BITS;
@@ -1709,6 +1729,7 @@ void build_desc(PassDesc &D, const PlanInput &in, const PassSpec &ps, bool inver
     D.stage_base = L.stage_base;
     D.f_nq = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / 4)));
     D.f_nchc = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / 32)));
+    D.f_nchc4 = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / 128)));
     D.f_nch = make_fdiv(static_cast<unsigned>((D.ax[1].E + 31) / 32));
     D.f_wpr = make_fdiv(static_cast<unsigned>(std::max(1, (D.ax[1].E / 32) * in.bits)));
     D.f_ngt = make_fdiv(static_cast<unsigned>(std::max(1, D.ax[1].E / in.group)));
