@@ -203,9 +203,14 @@ __device__ __forceinline__ void stage_row_fwht(float *xr, int s, int d, int part
     }
 }
 
+// HAD_ONLY: a build for processors whose every stage is all-Sylvester
+// (PolarQuant's H_128), carrying only the butterflies, so the hot loop's code
+// stays small (the general build's FMA stages of every width crowd the
+// instruction cache).
+template <bool HAD_ONLY>
 __device__ __forceinline__ void run_stage_row(float *xr, const float *C, const StageDev &S, int d, int part) {
     const int b = S.b, kp = S.kpad, s = static_cast<int>(S.s);
-    if (S.had) {
+    if (HAD_ONLY || S.had) {
         switch (b) {
             case 2: stage_row_fwht<2>(xr, s, d, part); return;
             case 4: stage_row_fwht<4>(xr, s, d, part); return;
@@ -215,6 +220,7 @@ __device__ __forceinline__ void run_stage_row(float *xr, const float *C, const S
             default: break;
         }
     }
+    if constexpr (HAD_ONLY) return;
     switch (b) {
         case 4: stage_row<4, true>(xr, C, b, kp, s, d, part); break;
         case 8: stage_row<8, true>(xr, C, b, kp, s, d, part); break;
@@ -357,7 +363,7 @@ __device__ __forceinline__ void store_codes(const float *X, int xp, int d, int64
     }
 }
 
-template <int MODE>
+template <int MODE, bool HAD_ONLY>
 __global__ void __launch_bounds__(NTT, 1)
 short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
     extern __shared__ float4 smem_f4[];
@@ -467,7 +473,7 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
         if (fwd) {
             int o = 0;
             for (int t = 0; t < P.m; ++t) {
-                if (mine) run_stage_row(xr, C + o, P.st[t], d, part);
+                if (mine) run_stage_row<HAD_ONLY>(xr, C + o, P.st[t], d, part);
                 __syncthreads();
                 o += static_cast<int>(d / P.st[t].b) * P.st[t].b * P.st[t].kpad;
             }
@@ -475,7 +481,7 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
             int o = Y.coef_total;
             for (int t = P.m - 1; t >= 0; --t) {
                 o -= static_cast<int>(d / P.st[t].b) * P.st[t].b * P.st[t].kpad;
-                if (mine) run_stage_row(xr, C + o, P.st[t], d, part);
+                if (mine) run_stage_row<HAD_ONLY>(xr, C + o, P.st[t], d, part);
                 __syncthreads();
             }
             if (mine) {
@@ -533,6 +539,21 @@ short_kernel(const PlanDev P, const QuantDev Q, const ShortLaunch L) {
     cp_async_wait_all();
 }
 
+template <bool H>
+const void *short_fn(int mode) {
+    return (mode == SHORT_FWD) ? reinterpret_cast<const void *>(short_kernel<SHORT_FWD, H>)
+         : (mode == SHORT_INV) ? reinterpret_cast<const void *>(short_kernel<SHORT_INV, H>)
+                               : reinterpret_cast<const void *>(short_kernel<SHORT_REQUANT, H>);
+}
+
+template <bool H>
+void short_run(int mode, unsigned grid, size_t smem, cudaStream_t st, const PlanDev &P, const QuantDev &q,
+               const ShortLaunch &L) {
+    if (mode == SHORT_FWD) short_kernel<SHORT_FWD, H><<<grid, NTT, smem, st>>>(P, q, L);
+    else if (mode == SHORT_INV) short_kernel<SHORT_INV, H><<<grid, NTT, smem, st>>>(P, q, L);
+    else short_kernel<SHORT_REQUANT, H><<<grid, NTT, smem, st>>>(P, q, L);
+}
+
 }  // namespace
 
 size_t short_smem_bytes(const PlanDev &P, int mode, int in_bits) {
@@ -552,9 +573,9 @@ int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &Lin, vo
     L.bins = (L.mode == SHORT_INV) ? 0 : (bins_exact(L.mode == SHORT_REQUANT ? L.q2 : q, 256) ? 1 : 0);
     const int in_bits = (L.mode == SHORT_FWD) ? 0 : q.bits;
     const size_t smem = short_smem_bytes(P, L.mode, in_bits);
-    const void *fn = (L.mode == SHORT_FWD) ? reinterpret_cast<const void *>(short_kernel<SHORT_FWD>)
-                   : (L.mode == SHORT_INV) ? reinterpret_cast<const void *>(short_kernel<SHORT_INV>)
-                                           : reinterpret_cast<const void *>(short_kernel<SHORT_REQUANT>);
+    bool had_only = true;            // every stage all-Sylvester: the butterfly-only build
+    for (int t = 0; t < P.m; ++t) had_only = had_only && P.st[t].had && P.st[t].b <= B_MAX;
+    const void *fn = had_only ? short_fn<true>(L.mode) : short_fn<false>(L.mode);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
@@ -566,9 +587,8 @@ int launch_short(const PlanDev &P, const QuantDev &q, const ShortLaunch &Lin, vo
     const int64_t ntiles = (L.nvec + ST - 1) / ST;
     const int64_t grid = ntiles < static_cast<int64_t>(sms) * per_sm ? ntiles : static_cast<int64_t>(sms) * per_sm;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (L.mode == SHORT_FWD) short_kernel<SHORT_FWD><<<static_cast<unsigned>(grid), NTT, smem, st>>>(P, q, L);
-    else if (L.mode == SHORT_INV) short_kernel<SHORT_INV><<<static_cast<unsigned>(grid), NTT, smem, st>>>(P, q, L);
-    else short_kernel<SHORT_REQUANT><<<static_cast<unsigned>(grid), NTT, smem, st>>>(P, q, L);
+    if (had_only) short_run<true>(L.mode, static_cast<unsigned>(grid), smem, st, P, q, L);
+    else short_run<false>(L.mode, static_cast<unsigned>(grid), smem, st, P, q, L);
     return cudaGetLastError();
 }
 

@@ -170,6 +170,34 @@ def test_two_sided_q5_takes_the_whole_vector_path():
     assert rel_l2(back.cpu().numpy(), ref_back) <= TOL_F32
 
 
+def test_short_vectors_mixed_sylvester_and_random_stages():
+    """A d = 128 right processor whose first stage is all-Sylvester (the
+    butterfly) and whose second has random orthogonal blocks (FMAs), with
+    signs: the general build of the short-vector kernel runs both stage
+    kinds; forward with the rotated copy and the inverse, against the
+    oracle's processor built from its own blocks of the same draws."""
+    torch.cuda.set_device(0)
+    radix, d, rows = (8, 16), 128, 300
+    g = synth.normal(111, 5, (d // 16) * 16 * 16).reshape(d // 16, 16, 16)
+    signs = synth.signs(112, 3, d)
+    plan = harp.Plan(radix, [harp.stage_blocks("hadamard", 8, d // 8), harp.stage_blocks("qr", 16, d // 16, gauss=g)],
+                     signs)
+    P = oracle.Processor(radix, [oracle.stage_blocks("hadamard", 8, d // 8),
+                                 oracle.stage_blocks("qr", 16, d // 16, gauss=g)], signs.astype(np.float64))
+    Wb = bf16_matrix(113, rows, d)
+    X = synth.bf16_bits_to_f64(Wb)
+    ref, oc, _, osc, m, sm = oracle.rotate_quantize(X, None, P, "lloyd_max", 4, 128)
+    cb = harp.Codebook("lloyd_max", 4, 128)
+    xb = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales, rot = harp.rotate_quantize(None, plan, cb, xb, want_rotated=True)
+    assert rel_l2(rot.cpu().numpy(), ref) <= TOL_F32
+    compare_quant(codes.cpu().numpy(), scales_np(scales), oc, osc, m, sm, 4, 128)
+    back = harp.dequantize_unrotate(None, plan, cb, codes, scales, rows, d, torch.float32)
+    ref_back = oracle.dequantize_unrotate(np_unpack(codes.cpu().numpy(), 4, d), scales_np(scales),
+                                          None, P, "lloyd_max", 4, 128)
+    assert rel_l2(back.cpu().numpy(), ref_back) <= TOL_F32
+
+
 @pytest.mark.parametrize("radix,bits,group", [((4, 8), 4, 32), ((8, 8), 3, 64), ((2, 16, 4), 2, 32)])
 def test_short_vectors_all_three_calls(radix, bits, group):
     """Rows of 32, 64 and 128 coordinates (one thread per row in the
