@@ -57,19 +57,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # L2 when a launch ends are counted by the next launch. When the pass-kernel
 # source differs from the captured one the figures no longer describe the
 # kernel and the roofline's traffic field is reported as null.
-MEASURED_TRAFFIC = {"kernel_src": "025b4495f0849231", "bytes": {
-    "fwd_p0_2bit": 49889024,
-    "fwd_p1_2bit": 86765824,
-    "fwd_p2_2bit": 68017152,
-    "inv_p0_2bit": 16860672,
-    "inv_p1_2bit": 86633984,
-    "inv_p2_2bit": 69223424,
-    "fwd_p0_4bit": 47279616,
-    "fwd_p1_4bit": 86482688,
-    "fwd_p2_4bit": 68010496,
-    "inv_p0_4bit": 21036032,
-    "inv_p1_4bit": 86616576,
-    "inv_p2_4bit": 69220096,
+MEASURED_TRAFFIC = {"kernel_src": "7a9a4395ad575c7d", "bytes": {
+    "fwd_p0_2bit": 50513920,
+    "fwd_p1_2bit": 87086848,
+    "fwd_p2_2bit": 67988480,
+    "inv_p0_2bit": 16457216,
+    "inv_p1_2bit": 87363584,
+    "inv_p2_2bit": 70016512,
+    "fwd_p0_4bit": 47332096,
+    "fwd_p1_4bit": 87085056,
+    "fwd_p2_4bit": 68019968,
+    "inv_p0_4bit": 21024256,
+    "inv_p1_4bit": 87330048,
+    "inv_p2_4bit": 69442304,
 }}
 PASS_SRC = os.path.join(ROOT, "rotation_preconditioned_bit_b200", "csrc", "harp_pass.cu")
 
