@@ -499,8 +499,10 @@ struct RowsGeom {
 };
 
 // Tile rows and shared-memory layout for d coordinates, or R = 0 when the
-// rows do not fit. R is a power of two, at most rmax and 64 / (largest
-// radix) so a thread's accumulators fit its registers.
+// rows do not fit. R is a power of two, at most rmax (<= 8) and 64 /
+// (largest radix) so a thread's accumulators fit its registers; R <= 8 also
+// keeps every row of a tile inside the block stages' loops (at most 8 rows
+// per thread).
 RowsGeom rows_geom(const PlanDev &P, int in_dtype, const QuantDev &q, int rmax = 8) {
     RowsGeom g{};
     const int d = static_cast<int>(P.d);
