@@ -317,37 +317,28 @@ def run_gpu(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    # ---- end to end through the public two-sided calls, host buffers
+    # ---- end to end through the C ABI's host-buffer calls
     e2e = None
     if not args.no_e2e:
         codes_h = [torch.empty(c.shape, dtype=c.dtype).pin_memory() for c, _ in outs]
         scales_h = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for _, s in outs]
-        outs_d = [out] + [torch.empty_like(out) for _ in cbs[1:]]
         outs_h = [torch.empty((ROWS, COLS), dtype=torch.bfloat16).pin_memory() for _ in cbs]
-        h2d = x_host.numel() * 2
-        d2h = sum(c.numel() + s.numel() * 2 + o.numel() * 2 for (c, s), o in zip(outs, outs_h))
-        ws_bytes = ws.numel() * 4
-        copy_stream = torch.cuda.Stream(dev)
+        # one device scratch (values, codes, scales, workspace) for every call,
+        # sized for the widest codes
+        scratch = max((harp.empty_host_scratch(left, right, cb, ROWS, COLS, harp.HARP_BF16, dev) for cb in cbs),
+                      key=lambda t: t.numel())
+        h2d = sum(x_host.numel() * 2 + c.numel() + s.numel() * 2 for c, s in zip(codes_h, scales_h))
+        d2h = sum(c.numel() + s.numel() * 2 + o.numel() * 2 for c, s, o in zip(codes_h, scales_h, outs_h))
+        ws_bytes = scratch.numel()
 
         def e2e_step():
-            # the library calls run in order on the compute stream; each
-            # result goes back to the host on a copy stream as soon as it is
-            # ready, so the copies overlap the next call
-            x.copy_(x_host, non_blocking=True)
-            for i, (cb, (codes, scales)) in enumerate(zip(cbs, outs)):
-                harp.harp_rotate_quantize(left, right, cb, x, codes, scales, None, ws, stream)
-                done_fwd = torch.cuda.Event()
-                done_fwd.record(stream)
-                harp.harp_dequantize_unrotate(left, right, cb, codes, scales, outs_d[i], ws, stream)
-                done_inv = torch.cuda.Event()
-                done_inv.record(stream)
-                with torch.cuda.stream(copy_stream):
-                    copy_stream.wait_event(done_fwd)
-                    codes_h[i].copy_(codes, non_blocking=True)
-                    scales_h[i].copy_(scales, non_blocking=True)
-                    copy_stream.wait_event(done_inv)
-                    outs_h[i].copy_(outs_d[i], non_blocking=True)
-            stream.wait_stream(copy_stream)
+            # per bit width: the forward from the host weight to host codes and
+            # scales, then the inverse from those host buffers to the host
+            # weight; copies and kernels in order on one stream
+            for i, cb in enumerate(cbs):
+                harp.harp_rotate_quantize_host(left, right, cb, x_host, codes_h[i], scales_h[i], scratch, stream)
+                harp.harp_dequantize_unrotate_host(left, right, cb, codes_h[i], scales_h[i], outs_h[i], scratch,
+                                                   stream)
 
         for _ in range(max(2, args.warmup)):
             e2e_step()
@@ -368,9 +359,9 @@ def run_gpu(args, rank, world, local_rank):
         e2e = {"value": round(job_gbs(world, args.steps, e_total), 2),
                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_total / args.steps, 4),
-               "api": "harp_rotate_quantize + harp_dequantize_unrotate (two-sided), pinned host buffers, "
-                      "device-to-host copies on a second stream overlapping the next call",
-               "workspace_bytes": ws_bytes}
+               "api": "harp_rotate_quantize_host + harp_dequantize_unrotate_host (two-sided): pinned host "
+                      "buffers in and out, every copy (cudaMemcpyAsync) and kernel in order on one stream",
+               "scratch_bytes": ws_bytes}
     del flush
     return total_ms, step_ms, kt, clk, e2e, npass, pass_fma, alt
 

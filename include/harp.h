@@ -310,6 +310,44 @@ int harp_dequantize_unrotate(harp_plan_t left, harp_plan_t right, harp_codebook_
                              int64_t cols, void *out, int out_dtype, void *workspace,
                              size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------ host-buffer variants */
+
+/* The fused calls for callers whose data live in host memory: each copies
+ * its inputs from host buffers into a caller-provided device scratch,
+ * runs the device call there, and copies its outputs back into host
+ * buffers. Copies (one cudaMemcpyAsync per buffer) and kernels are ordered
+ * on `stream` and the call returns once they are enqueued: the host buffers
+ * must stay valid and unchanged until the stream has passed them
+ * (synchronise the stream before reading the outputs). Pinned (page-locked)
+ * host buffers make the copies asynchronous; pageable ones also work, with
+ * the CUDA runtime's staging. Nothing is allocated.
+ *
+ * Scratch layout (each part 256-byte aligned): values (rows*cols elements
+ * of the value dtype: the input of the forward, the output of the inverse),
+ * packed codes, fp16 scales, then the workspace of harp_workspace_size.
+ * harp_host_scratch_size gives the bytes for a call's shapes and value
+ * dtype (HARP_BF16 or HARP_F32). Errors: those of the device call, plus
+ * INVALID_ARG (NULL host buffer with rows, cols > 0; value dtype not bf16 /
+ * f32) and WORKSPACE (dev_scratch NULL or smaller than the size). */
+int harp_host_scratch_size(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int64_t rows,
+                           int64_t cols, int value_dtype, size_t *bytes);
+
+/* harp_rotate_quantize with host `in` (rows x cols, in_dtype, row-major) and
+ * host outputs `codes` (rows * cols * bits / 8 bytes) and `scales`
+ * (rows * cols / group fp16 values)  [HARP 3; PolarQuant 2]. */
+int harp_rotate_quantize_host(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,
+                              const void *in, int in_dtype, int64_t rows, int64_t cols,
+                              uint8_t *codes, uint16_t *scales, void *dev_scratch,
+                              size_t scratch_bytes, void *stream);
+
+/* harp_dequantize_unrotate with host `codes` and `scales` and host output
+ * `out` (rows x cols, out_dtype HARP_BF16 or HARP_F32)  [PolarQuant 2;
+ * HARP 5]. */
+int harp_dequantize_unrotate_host(harp_plan_t left, harp_plan_t right, harp_codebook_t cb,
+                                  const uint8_t *codes, const uint16_t *scales, int64_t rows,
+                                  int64_t cols, void *out, int out_dtype, void *dev_scratch,
+                                  size_t scratch_bytes, void *stream);
+
 /* ------------------------------------------------------------ timing hooks */
 
 /* Number of kernel launches (passes) harp_rotate_quantize and

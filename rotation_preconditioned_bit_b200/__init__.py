@@ -41,7 +41,8 @@ EXPORTS = (
     "harp_rotate_quantize", "harp_dequantize_unrotate", "harp_rotate_quantize_static",
     "harp_pass_count", "harp_pass_fma", "harp_set_pass_events",
     "harp_theta_blocks", "harp_plan_load_theta", "harp_requantize", "harp_fault_status",
-    "harp_set_block_stages",
+    "harp_set_block_stages", "harp_host_scratch_size", "harp_rotate_quantize_host",
+    "harp_dequantize_unrotate_host",
 )
 
 
@@ -94,6 +95,10 @@ def lib():
         L.harp_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _INT, _P, _P, _P, _P, _P]
         L.harp_fault_status.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.harp_set_block_stages.argtypes = [_INT]
+        L.harp_host_scratch_size.argtypes = [_P, _P, _P, _I64, _I64, _INT, ctypes.POINTER(ctypes.c_size_t)]
+        L.harp_rotate_quantize_host.argtypes = [_P, _P, _P, _P, _INT, _I64, _I64, _P, _P, _P, ctypes.c_size_t, _P]
+        L.harp_dequantize_unrotate_host.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _P, _INT, _P,
+                                                    ctypes.c_size_t, _P]
         _lib = L
     return _lib
 
@@ -414,6 +419,56 @@ def harp_dequantize_unrotate(left, right, cb, codes, scales, out, workspace=None
 
 
 # ------------------------------------------------------------ allocating wrappers
+
+def _require_host(*ts):
+    for t in ts:
+        if t is not None and t.is_cuda:
+            raise ValueError("the _host calls take CPU (preferably pinned) tensors for their host buffers")
+
+
+def harp_host_scratch_size(left, right, cb, rows, cols, value_dtype) -> int:
+    """Device scratch bytes of harp_rotate_quantize_host /
+    harp_dequantize_unrotate_host for these shapes and value dtype."""
+    n = ctypes.c_size_t()
+    _check(lib().harp_host_scratch_size(left.handle if left else None, right.handle, cb.handle, rows, cols,
+                                        int(value_dtype), ctypes.byref(n)), "harp_host_scratch_size")
+    return n.value
+
+
+def empty_host_scratch(left, right, cb, rows, cols, value_dtype, device="cuda"):
+    import torch
+    n = harp_host_scratch_size(left, right, cb, rows, cols, value_dtype)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+
+
+def harp_rotate_quantize_host(left, right, cb, x, codes, scales, scratch, stream=None):
+    """harp_rotate_quantize on host buffers: x, codes and scales are CPU
+    tensors (pinned for asynchronous copies), scratch a CUDA byte tensor of
+    harp_host_scratch_size bytes. Enqueued on the stream; synchronise it
+    before reading codes and scales."""
+    _require_host(x, codes, scales)
+    _require_cuda(scratch)
+    rows, cols = x.shape
+    _check(lib().harp_rotate_quantize_host(left.handle if left else None, right.handle, cb.handle, _ptr(x),
+                                           _dtype_code(x), rows, cols, _ptr(codes), _ptr(scales), _ptr(scratch),
+                                           scratch.numel() * scratch.element_size(), _stream(stream)),
+           "harp_rotate_quantize_host")
+    return codes, scales
+
+
+def harp_dequantize_unrotate_host(left, right, cb, codes, scales, out, scratch, stream=None):
+    """harp_dequantize_unrotate on host buffers (codes, scales, out CPU
+    tensors; out bf16 or fp32 [rows, cols]); enqueued on the stream."""
+    _require_host(codes, scales, out)
+    _require_cuda(scratch)
+    rows, cols = out.shape
+    _check(lib().harp_dequantize_unrotate_host(left.handle if left else None, right.handle, cb.handle,
+                                               _ptr(codes), _ptr(scales), rows, cols, _ptr(out), _dtype_code(out),
+                                               _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                               _stream(stream)),
+           "harp_dequantize_unrotate_host")
+    return out
+
 
 def empty_codes(rows, cols, cb, device="cuda"):
     import torch

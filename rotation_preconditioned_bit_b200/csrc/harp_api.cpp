@@ -774,6 +774,105 @@ int harp_pass_fma(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int p
     return HARP_OK;
 }
 
+// ------------------------------------------------------------ host-buffer variants
+
+namespace {
+
+size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+struct HostScratch {
+    size_t values, codes, scales, ws, total;   // byte offsets of the parts, total bytes
+    size_t value_bytes, code_bytes, scale_bytes, ws_bytes;
+};
+
+int host_scratch(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int64_t rows, int64_t cols,
+                 int value_dtype, HostScratch &h) {
+    if (!right || !cb || rows < 0 || cols < 0) return HARP_ERR_INVALID_ARG;
+    if (value_dtype != HARP_BF16 && value_dtype != HARP_F32) return HARP_ERR_INVALID_ARG;
+    size_t ws = 0;
+    int st = harp_workspace_size(left, right, rows, cols, &ws);
+    if (st) return st;
+    const size_t n = static_cast<size_t>(rows) * static_cast<size_t>(cols);
+    h.value_bytes = n * (value_dtype == HARP_BF16 ? 2 : 4);
+    h.code_bytes = n * static_cast<size_t>(cb->q.bits) / 8;
+    h.scale_bytes = (cb->q.group > 0 ? n / static_cast<size_t>(cb->q.group) : 0) * 2;
+    h.ws_bytes = ws;
+    h.values = 0;
+    h.codes = align256(h.value_bytes);
+    h.scales = h.codes + align256(h.code_bytes);
+    h.ws = h.scales + align256(h.scale_bytes);
+    h.total = h.ws + ws;
+    return HARP_OK;
+}
+
+}  // namespace
+
+int harp_host_scratch_size(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, int64_t rows,
+                           int64_t cols, int value_dtype, size_t *bytes) {
+    if (!bytes) return HARP_ERR_INVALID_ARG;
+    HostScratch h{};
+    const int st = host_scratch(left, right, cb, rows, cols, value_dtype, h);
+    if (st) return st;
+    *bytes = h.total;
+    return HARP_OK;
+}
+
+int harp_rotate_quantize_host(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, const void *in,
+                              int in_dtype, int64_t rows, int64_t cols, uint8_t *codes, uint16_t *scales,
+                              void *dev_scratch, size_t scratch_bytes, void *stream) {
+    HostScratch h{};
+    int st = host_scratch(left, right, cb, rows, cols, in_dtype, h);
+    if (st) return st;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!in || !codes || !scales) return HARP_ERR_INVALID_ARG;
+    if (!dev_scratch || scratch_bytes < h.total) return HARP_ERR_WORKSPACE;
+    if (!aligned(dev_scratch, 256)) return HARP_ERR_ALIGNMENT;
+    char *base = static_cast<char *>(dev_scratch);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(base + h.values, in, h.value_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess) {
+        cudaGetLastError();
+        return HARP_ERR_CUDA;
+    }
+    st = harp_rotate_quantize(left, right, cb, base + h.values, in_dtype, rows, cols,
+                              reinterpret_cast<uint8_t *>(base + h.codes), reinterpret_cast<uint16_t *>(base + h.scales),
+                              nullptr, h.ws_bytes ? base + h.ws : nullptr, h.ws_bytes, stream);
+    if (st) return st;
+    if (cudaMemcpyAsync(codes, base + h.codes, h.code_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+        cudaMemcpyAsync(scales, base + h.scales, h.scale_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess) {
+        cudaGetLastError();
+        return HARP_ERR_CUDA;
+    }
+    return HARP_OK;
+}
+
+int harp_dequantize_unrotate_host(harp_plan_t left, harp_plan_t right, harp_codebook_t cb, const uint8_t *codes,
+                                  const uint16_t *scales, int64_t rows, int64_t cols, void *out, int out_dtype,
+                                  void *dev_scratch, size_t scratch_bytes, void *stream) {
+    HostScratch h{};
+    int st = host_scratch(left, right, cb, rows, cols, out_dtype, h);
+    if (st) return st;
+    if (rows == 0 || cols == 0) return HARP_OK;
+    if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
+    if (!dev_scratch || scratch_bytes < h.total) return HARP_ERR_WORKSPACE;
+    if (!aligned(dev_scratch, 256)) return HARP_ERR_ALIGNMENT;
+    char *base = static_cast<char *>(dev_scratch);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(base + h.codes, codes, h.code_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(base + h.scales, scales, h.scale_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess) {
+        cudaGetLastError();
+        return HARP_ERR_CUDA;
+    }
+    st = harp_dequantize_unrotate(left, right, cb, reinterpret_cast<const uint8_t *>(base + h.codes),
+                                  reinterpret_cast<const uint16_t *>(base + h.scales), rows, cols, base + h.values,
+                                  out_dtype, h.ws_bytes ? base + h.ws : nullptr, h.ws_bytes, stream);
+    if (st) return st;
+    if (cudaMemcpyAsync(out, base + h.values, h.value_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess) {
+        cudaGetLastError();
+        return HARP_ERR_CUDA;
+    }
+    return HARP_OK;
+}
+
 int harp_set_block_stages(int mode) {
     if (mode < HARP_BLOCK_STAGES_AUTO || mode > HARP_BLOCK_STAGES_FFMA) return HARP_ERR_INVALID_ARG;
     harp::set_block_stages(mode);

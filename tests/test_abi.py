@@ -165,6 +165,38 @@ def test_compute_calls_reject_bad_arguments_before_launch():
     assert L.harp_workspace_size(ctypes.c_void_p(8), None, 10, 20, ctypes.byref(n)) == 0 and n.value == 1600
 
 
+def test_host_buffer_calls_scratch_size_and_checks():
+    """The host-buffer variants: scratch = values + codes + scales (+ the
+    two-sided workspace), each part 256-byte aligned; argument errors come
+    back before anything is copied or launched."""
+    L = harp.lib()
+    cb = harp.Codebook("lloyd_max", 3, 128)
+    fake = ctypes.c_void_p(8)
+    n = ctypes.c_size_t()
+    # right-only, bf16 values: 64*256*2 + 64*256*3/8 + 64*2*2 bytes
+    assert L.harp_host_scratch_size(None, fake, cb.handle, 64, 256, harp.HARP_BF16, ctypes.byref(n)) == 0
+    assert n.value == 32768 + 6144 + 256
+    # two-sided, fp32 values: plus rows*cols*8 bytes of workspace
+    assert L.harp_host_scratch_size(fake, fake, cb.handle, 64, 256, harp.HARP_F32, ctypes.byref(n)) == 0
+    assert n.value == 65536 + 6144 + 256 + 131072
+    assert L.harp_host_scratch_size(None, None, cb.handle, 64, 256, harp.HARP_BF16, ctypes.byref(n)) == 1
+    assert L.harp_host_scratch_size(None, fake, cb.handle, 64, 256, 2, ctypes.byref(n)) == 1   # f16 values
+    assert L.harp_host_scratch_size(None, fake, cb.handle, 64, 256, harp.HARP_BF16, None) == 1
+    # empty: nothing to do; missing or short scratch; missing host buffers
+    assert L.harp_rotate_quantize_host(None, fake, cb.handle, None, harp.HARP_BF16, 0, 256, None, None,
+                                       None, 0, None) == 0
+    assert L.harp_rotate_quantize_host(None, fake, cb.handle, fake, harp.HARP_BF16, 64, 256, fake, fake,
+                                       None, 0, None) == 5
+    assert L.harp_rotate_quantize_host(None, fake, cb.handle, fake, harp.HARP_BF16, 64, 256, fake, fake,
+                                       ctypes.c_void_p(4096), 1024, None) == 5
+    assert L.harp_rotate_quantize_host(None, fake, cb.handle, None, harp.HARP_BF16, 64, 256, fake, fake,
+                                       ctypes.c_void_p(4096), 1 << 20, None) == 1
+    assert L.harp_dequantize_unrotate_host(None, fake, cb.handle, fake, fake, 64, 256, None, harp.HARP_BF16,
+                                           ctypes.c_void_p(4096), 1 << 20, None) == 1
+    assert L.harp_dequantize_unrotate_host(None, fake, cb.handle, fake, fake, 64, 256, fake, harp.HARP_F16,
+                                           ctypes.c_void_p(4096), 1 << 20, None) == 1
+
+
 def test_theta_calls_reject_bad_arguments_before_launch():
     L = harp.lib()
     fake = ctypes.c_void_p(4096)
