@@ -323,22 +323,32 @@ def run_gpu(args, rank, world, local_rank):
         codes_h = [torch.empty(c.shape, dtype=c.dtype).pin_memory() for c, _ in outs]
         scales_h = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for _, s in outs]
         outs_h = [torch.empty((ROWS, COLS), dtype=torch.bfloat16).pin_memory() for _ in cbs]
-        # one device scratch (values, codes, scales, workspace) for every call,
-        # sized for the widest codes
-        scratch = max((harp.empty_host_scratch(left, right, cb, ROWS, COLS, harp.HARP_BF16, dev) for cb in cbs),
-                      key=lambda t: t.numel())
+        # the two bit widths are independent chains: each runs on its own
+        # stream with its own device scratch (values, codes, scales,
+        # workspace), so one chain's PCIe copies overlap the other's kernels
+        streams = [stream] + [torch.cuda.Stream(dev) for _ in cbs[1:]]
+        scratches = [harp.empty_host_scratch(left, right, cb, ROWS, COLS, harp.HARP_BF16, dev) for cb in cbs]
         h2d = sum(x_host.numel() * 2 + c.numel() + s.numel() * 2 for c, s in zip(codes_h, scales_h))
         d2h = sum(c.numel() + s.numel() * 2 + o.numel() * 2 for c, s, o in zip(codes_h, scales_h, outs_h))
-        ws_bytes = scratch.numel()
+        ws_bytes = sum(t.numel() for t in scratches)
 
         def e2e_step():
             # per bit width: the forward from the host weight to host codes and
             # scales, then the inverse from those host buffers to the host
-            # weight; copies and kernels in order on one stream
+            # weight, in order on that chain's stream
+            start = torch.cuda.Event()
+            start.record(stream)
             for i, cb in enumerate(cbs):
-                harp.harp_rotate_quantize_host(left, right, cb, x_host, codes_h[i], scales_h[i], scratch, stream)
-                harp.harp_dequantize_unrotate_host(left, right, cb, codes_h[i], scales_h[i], outs_h[i], scratch,
-                                                   stream)
+                st = streams[i]
+                if st is not stream:
+                    st.wait_event(start)
+                harp.harp_rotate_quantize_host(left, right, cb, x_host, codes_h[i], scales_h[i], scratches[i], st)
+                harp.harp_dequantize_unrotate_host(left, right, cb, codes_h[i], scales_h[i], outs_h[i],
+                                                   scratches[i], st)
+            for st in streams[1:]:
+                done = torch.cuda.Event()
+                done.record(st)
+                stream.wait_event(done)
 
         for _ in range(max(2, args.warmup)):
             e2e_step()
@@ -360,7 +370,8 @@ def run_gpu(args, rank, world, local_rank):
                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_total / args.steps, 4),
                "api": "harp_rotate_quantize_host + harp_dequantize_unrotate_host (two-sided): pinned host "
-                      "buffers in and out, every copy (cudaMemcpyAsync) and kernel in order on one stream",
+                      "buffers in and out; per bit width one stream, copies (cudaMemcpyAsync) and kernels in "
+                      "order on it, the two widths' streams concurrent",
                "scratch_bytes": ws_bytes}
     del flush
     return total_ms, step_ms, kt, clk, e2e, npass, pass_fma, alt
