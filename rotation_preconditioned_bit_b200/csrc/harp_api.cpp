@@ -827,6 +827,7 @@ int harp_rotate_quantize_host(harp_plan_t left, harp_plan_t right, harp_codebook
     if (!in || !codes || !scales) return HARP_ERR_INVALID_ARG;
     if (!dev_scratch || scratch_bytes < h.total) return HARP_ERR_WORKSPACE;
     if (!aligned(dev_scratch, 256)) return HARP_ERR_ALIGNMENT;
+    if (int dv = plans_on_current_device(left, right)) return dv;   // before anything is copied
     char *base = static_cast<char *>(dev_scratch);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (cudaMemcpyAsync(base + h.values, in, h.value_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess) {
@@ -855,6 +856,7 @@ int harp_dequantize_unrotate_host(harp_plan_t left, harp_plan_t right, harp_code
     if (!out || !codes || !scales) return HARP_ERR_INVALID_ARG;
     if (!dev_scratch || scratch_bytes < h.total) return HARP_ERR_WORKSPACE;
     if (!aligned(dev_scratch, 256)) return HARP_ERR_ALIGNMENT;
+    if (int dv = plans_on_current_device(left, right)) return dv;   // before anything is copied
     char *base = static_cast<char *>(dev_scratch);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (cudaMemcpyAsync(base + h.codes, codes, h.code_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
