@@ -68,6 +68,7 @@ struct RowsDesc {
     uint8_t *codes;
     uint16_t *scales;
     int chunk;                    // coordinates per quantiser chunk (32 x CW)
+    int fuse0;                    // stage 0 reads the staged input itself (register-block radix, not Sylvester)
     int stage_base, part_base, bar_base, lev_base;   // float offsets in shared memory
 };
 
@@ -219,6 +220,87 @@ __device__ __forceinline__ void stage_rows_rc(float *T, const RowsDesc &D, int t
             }
         }
     }
+}
+
+// Stage 0 of a register-block processor straight from the staged input
+// rows (bf16 or fp32, row-major, d per row): x_j = input * sign (the signs of
+// the thread's group held in registers), outputs into the fp32 tile; the
+// separate convert step is skipped. Same thread <-> (group, rows) map and
+// arithmetic as stage_rows_rc.
+template <int B, int RT>
+__device__ __forceinline__ void stage0_from_input(const void *S, float *T, const RowsDesc &D, int nrows, int tid) {
+    static_assert(B == 2 || B == 4 || B == 8, "register-resident blocks take radices 2, 4 and 8");
+    const int s = D.s[0], sl = D.sl[0], kq = D.kpad[0] >> 2, d = D.d;
+    const int G = d / B;
+    const int GT = G < RT_THREADS ? G : RT_THREADS;
+    const int RS = RT_THREADS / GT;
+    const int rs = tid / GT;
+    if (rs >= RS) return;
+    const int pitch = D.pitch;
+    for (int g = tid - rs * GT; g < G; g += GT) {
+        const int h = g >> sl, l = g & (s - 1);
+        const int base = h * B * s + l;
+        const float4 *cp = reinterpret_cast<const float4 *>(D.gfwd[0]) + g;
+        f2_t cc[B][B / 2];
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+#pragma unroll
+            for (int q = 0; q < (B + 3) / 4; ++q) {
+                const float4 v = __ldg(cp + static_cast<int64_t>(j * kq + q) * G);
+                cc[j][2 * q] = f2_pack(v.x, v.y);
+                if constexpr (B >= 4) cc[j][2 * q + 1] = f2_pack(v.z, v.w);
+            }
+        }
+        int xa[B];
+        float sg[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+            xa[j] = sk(base + j * s);
+            sg[j] = __ldg(D.signs + base + j * s);
+        }
+#pragma unroll 2
+        for (int i = 0; i < RT; ++i) {
+            const int r = rs + i * RS;
+            if (r >= nrows) break;
+            float x[B];
+            if (D.in_bf16) {
+                const unsigned short *src = static_cast<const unsigned short *>(S) + r * d + base;
+#pragma unroll
+                for (int j = 0; j < B; ++j) x[j] = __uint_as_float(static_cast<unsigned>(src[j * s]) << 16) * sg[j];
+            } else {
+                const float *src = static_cast<const float *>(S) + r * d + base;
+#pragma unroll
+                for (int j = 0; j < B; ++j) x[j] = src[j * s] * sg[j];
+            }
+            f2_t acc[B / 2];
+#pragma unroll
+            for (int q = 0; q < B / 2; ++q) acc[q] = 0ull;
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                const f2_t xd = f2_pack(x[j], x[j]);
+#pragma unroll
+                for (int q = 0; q < B / 2; ++q) acc[q] = f2_fma(cc[j][q], xd, acc[q]);
+            }
+            float *row = T + r * pitch;
+#pragma unroll
+            for (int q = 0; q < B / 2; ++q) {
+                float y0, y1;
+                f2_unpack(acc[q], y0, y1);
+                row[xa[2 * q]] = y0;
+                row[xa[2 * q + 1]] = y1;
+            }
+        }
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void stage0_from_input_any(const void *S, float *T, const RowsDesc &D, int nrows, int tid) {
+    const int G = D.d / B;
+    const int GT = G < RT_THREADS ? G : RT_THREADS;
+    const int rt = (D.R + RT_THREADS / GT - 1) / (RT_THREADS / GT);
+    if (rt <= 2) stage0_from_input<B, 2>(S, T, D, nrows, tid);
+    else if (rt <= 4) stage0_from_input<B, 4>(S, T, D, nrows, tid);
+    else stage0_from_input<B, 8>(S, T, D, nrows, tid);
 }
 
 // A stage whose blocks are all the normalised Sylvester Hadamard matrix H_b
@@ -456,12 +538,20 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rows_kernel(const __grid_consta
             if (tid == 0) atomicOr(&g_rows_fault, 4u);
             break;
         }
-        convert_rows(D, S, T, nrows, tid);
+        if (D.fuse0) {
+            switch (D.b[0]) {
+                case 2: stage0_from_input_any<2>(S, T, D, nrows, tid); break;
+                case 4: stage0_from_input_any<4>(S, T, D, nrows, tid); break;
+                default: stage0_from_input_any<8>(S, T, D, nrows, tid); break;
+            }
+        } else {
+            convert_rows(D, S, T, nrows, tid);
+        }
         // the staging buffer's reads are ordered before the next bulk copy into it
         tc::fence_proxy_async();
         __syncthreads();
         if (tid == 0 && t + gridDim.x < ntiles) issue(t + gridDim.x);
-        for (int st = 0; st < D.m; ++st) {
+        for (int st = D.fuse0 ? 1 : 0; st < D.m; ++st) {
             if (D.had[st]) {
                 switch (D.b[st]) {
                     case 2: stage_rows_fwht<2>(T, D, st, nrows, tid); break;
@@ -584,6 +674,7 @@ int launch_rows(const PlanDev &P, const QuantDev &q, const void *in, int in_dtyp
     D.codes = codes;
     D.scales = scales;
     D.chunk = g.chunk;
+    D.fuse0 = (P.st[0].b <= 8 && !P.st[0].had) ? 1 : 0;
     D.stage_base = g.stage_base;
     D.part_base = g.part_base;
     D.lev_base = g.lev_base;
